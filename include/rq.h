@@ -1,0 +1,199 @@
+/*
+ * rq.h -- C ABI of the rotated W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer is y = Q_a(R x) . Q_w(W R^T)^T (+ c . L^T):
+ *   - R is a randomized permuted block-Hadamard (RPBH) rotation: random signs,
+ *     one fixed permutation of the K input channels, then an orthonormal
+ *     Walsh-Hadamard transform per block of `block` channels (OrbitQuant
+ *     abstract, "randomized permuted block-Hadamard"; TR-DQ: Time-Rotation
+ *     Diffusion Quantization, section 3.2, Eq. 8, block-diagonal rotation).
+ *   - The weight side W R^T is folded and quantized offline, so the rotation
+ *     cancels inside the layer and only R x runs online (OrbitQuant abstract;
+ *     TR-DQ Eq. 9).
+ *   - Q is one of: symmetric uniform INT4 (TR-DQ section 3.1, Eq. 1-3, absmax
+ *     form), a Lloyd-Max codebook for the marginal of a rotated coordinate after
+ *     per-token normalisation (OrbitQuant abstract), or NVFP4 (E2M1 elements with
+ *     a UE4M3 scale per 16 elements; DiRotQ abstract, NVFP4 on Blackwell).
+ *   - c . L^T is the optional DiRotQ low-rank branch: r PCA coefficients of the
+ *     activation kept in BF16 (DiRotQ abstract).
+ *
+ * Conventions for every call
+ *   - All buffers are owned by the caller.  No call allocates device memory or
+ *     keeps a pointer after it returns.
+ *   - "device" pointers must be device-accessible global memory of the current
+ *     CUDA device, 16-byte aligned; "host" pointers are ordinary host memory
+ *     read or written before the call returns.
+ *   - Device work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
+ *     stream) and is asynchronous to the host.
+ *   - BF16 tensors are passed as their 16-bit patterns (uint16_t).
+ *   - Matrices are row-major.  Packed 4-bit codes store element 2j in bits 0-3
+ *     and element 2j+1 in bits 4-7 of byte j of the row; packed 2-bit codes store
+ *     element 4j+i in bits 2i..2i+1 of byte j.
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     return RQ_ERR_INVALID_ARG / RQ_ERR_UNSUPPORTED / RQ_ERR_ALIGNMENT with a
+ *     message for rq_last_error().  A failed launch returns RQ_ERR_CUDA.
+ *   - `status` (device int32, caller-initialised to 0) receives a non-zero code
+ *     if a kernel gave up a bounded wait; read it back with rq_read_status().
+ *     Kernels never wait without bound.
+ */
+#ifndef RQ_H_
+#define RQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t rq_status;
+#define RQ_OK 0
+#define RQ_ERR_INVALID_ARG 1
+#define RQ_ERR_UNSUPPORTED 2
+#define RQ_ERR_ALIGNMENT 3
+#define RQ_ERR_CUDA 4
+#define RQ_ERR_TIMEOUT 5
+
+/* Quantization formats. */
+#define RQ_INT4 1  /* symmetric INT4 in -7..7, two's-complement nibbles          */
+#define RQ_LM16 2  /* 16-level Lloyd-Max codebook index, nibbles                  */
+#define RQ_NVFP4 3 /* E2M1 nibbles + UE4M3 block scale per 16 + FP32 row scale    */
+#define RQ_LM4 4   /* 4-level Lloyd-Max codebook index, 2-bit (weights only)       */
+
+/*
+ * rq_make_rotation -- host.  Draw the RPBH rotation for K channels.
+ *   Source: OrbitQuant abstract ("randomized permuted block-Hadamard (RPBH)
+ *   rotation"); TR-DQ section 3.2 (a permutation is an orthogonal matrix;
+ *   Eq. 8 block-diagonal structure with K / block blocks).
+ *   K      number of input channels, K % block == 0.
+ *   block  Hadamard block size, a power of two, 128 <= block <= 512 for the
+ *          device calls (any power of two >= 2 here).
+ *   seed   64-bit seed of the SplitMix64 stream: K sign draws first (negative
+ *          when bit 63 is set), then a Fisher-Yates shuffle of 0..K-1 from the
+ *          top index down with unbiased rejection draws.
+ *   sign   [out, host, K] int8 +1/-1 per input channel (may be NULL).
+ *   perm   [out, host, K] int32: output position i reads channel perm[i] (may be NULL).
+ *   rot    [out, host, K] int32 signed permutation: bits 0-30 = perm[i], bit 31
+ *          set when sign[perm[i]] < 0.  This is the table the device calls
+ *          take (copy it to device memory).  May be NULL.
+ *   R x is then y_i = (1/sqrt(block)) sum_j H[i mod block][j mod block]
+ *   sign[perm[j]] x[perm[j]] over j in the block of i.
+ */
+rq_status rq_make_rotation(int32_t K, int32_t block, uint64_t seed, int8_t* sign, int32_t* perm, int32_t* rot);
+
+/*
+ * rq_make_codebook -- host.  Lloyd-Max quantizer for the marginal of one
+ * coordinate of a rotated row normalised to norm sqrt(K):
+ * f(u) ~ (1 - u^2/K)^((K-3)/2) on |u| < sqrt(K) (OrbitQuant abstract: after RPBH
+ * every coordinate follows one known marginal, so one Lloyd-Max codebook serves
+ * all inputs of a given dimension).  FP64 Lloyd iteration (centroid = conditional
+ * mean, boundary = midpoint) on the symmetric density until no value moves by
+ * 1e-13.
+ *   K       input dimension (>= 4).    levels  4 or 16.
+ *   centroids       [out, host, levels] FP64, ascending (may be NULL)
+ *   boundaries      [out, host, levels-1] FP64 (may be NULL)
+ *   boundaries_f32  [out, host, levels-1] FP32 rounding of the boundaries: the
+ *                   table the quantizer compares against (may be NULL)
+ *   centroids_e4m3  [out, host, levels] E4M3 bytes of the FP32-rounded
+ *                   centroids: the values the FP8 GEMM multiplies (may be NULL)
+ */
+rq_status rq_make_codebook(int32_t K, int32_t levels, double* centroids, double* boundaries,
+                           float* boundaries_f32, uint8_t* centroids_e4m3);
+
+/*
+ * rq_pca_basis -- host.  Top-r eigenvectors of the uncentered second moment
+ * X^T X / n of n calibration tokens (DiRotQ abstract: a low-rank subspace of
+ * dominant activation variance via PCA), FP64 Jacobi eigen-solver on the n x n
+ * Gram matrix, each vector's largest-magnitude entry made positive.
+ *   calib  [in, host, n x K] BF16 bits.   n >= r, 1 <= r <= 64.
+ *   U      [out, host, K x r] BF16 bits (column j = eigenvector j).
+ *   eigenvalues [out, host, r] FP64, descending (may be NULL).
+ */
+rq_status rq_pca_basis(const uint16_t* calib, int32_t n, int32_t K, int32_t r, uint16_t* U, double* eigenvalues);
+
+/*
+ * rq_rotate_quantize_act -- device, async.  The online activation transform:
+ * rotate each row of X with R, normalise per token, quantize, pack.
+ * (OrbitQuant abstract: only a forward rotation on the activations remains at
+ * run time; TR-DQ section 3.2: dynamic per-token ranges computed online.)
+ *   fmt    RQ_INT4 | RQ_LM16 | RQ_NVFP4.
+ *   X      [device, M x K] BF16.     M >= 1.  K % block == 0, K <= 16384,
+ *          K % 128 == 0 (INT4 / LM16), K % 256 == 0 (NVFP4).
+ *   rot    [device, K] signed permutation from rq_make_rotation.
+ *   boundaries [host, levels-1] FP32 codebook boundaries (RQ_LM16), else NULL.
+ *   U, r   [device, K x r] BF16 PCA basis and its rank (r == 32), or NULL / 0.
+ *          With U: c = bf16(x U) (FP32, sequential over k) is written to c_out
+ *          and the residual x - c U^T is what gets rotated and quantized.
+ *   c_out  [device, M x r] BF16 or NULL.
+ *   codes  [device, M x K/2] packed nibbles.
+ *   scale  [device, M] FP32 per-token scale: amax/7 (INT4), ||y||/sqrt(K)
+ *          (codebook), amax/2688 (NVFP4).
+ *   block_scale [device] NVFP4 only: UE4M3 scale per 16 elements in 128-row x
+ *          64-column tiles of 512 bytes, tile (mt, kt) at (mt*(K/64)+kt)*512, entry
+ *          (m, kb) inside at (m%32)*16 + ((m%128)/32)*4 + kb%4; size
+ *          ceil(M/128)*128*(K/16) bytes.  Padding rows are never read as data.
+ *   status [device] int32 error word (see above).
+ */
+rq_status rq_rotate_quantize_act(int32_t fmt, const uint16_t* X, int32_t M, int32_t K, int32_t block,
+                                 const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r,
+                                 uint16_t* c_out, uint8_t* codes, float* scale, uint8_t* block_scale,
+                                 int32_t* status, void* stream);
+
+/*
+ * rq_quantize_weights -- device, async.  Offline weight preparation: every row
+ * w_n of W becomes R w_n (the row of W R^T) and is quantized with the same
+ * procedure (OrbitQuant abstract: the same quantizer extended to weight rows,
+ * the rotation absorbed into the weights).
+ *   fmt    RQ_INT4 (one scale per 128 rotated coordinates) | RQ_LM16 | RQ_LM4 |
+ *          RQ_NVFP4.
+ *   W      [device, N x K] BF16.
+ *   U, r, L_out  optional: L = bf16(W U) [device, N x r] for the low-rank branch
+ *          (the full row is still what gets quantized).
+ *   codes  [device, N x K/2] (RQ_LM4: N x K/4).
+ *   scale  [device] RQ_INT4: [K/128][N] group-major; otherwise [N].
+ *   block_scale  NVFP4 only, same layout as for activations with N rows.
+ */
+rq_status rq_quantize_weights(int32_t fmt, const uint16_t* W, int32_t N, int32_t K, int32_t block,
+                              const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r,
+                              uint16_t* L_out, uint8_t* codes, float* scale, uint8_t* block_scale,
+                              int32_t* status, void* stream);
+
+/*
+ * rq_w4a4_linear -- device, async.  The 4-bit x 4-bit GEMM on rotated codes with
+ * per-token x per-group (INT4) or per-token x per-row scales, plus the optional
+ * low-rank term (OrbitQuant abstract: the rotation cancels inside each linear
+ * layer; DiRotQ abstract: a 4-bit GEMM plus a thin rank-r GEMM):
+ *   Y[m, n] = a_scale[m] * sum_g w_scale[g, n] * sum_{k in g} a(m, k) w(n, k)
+ *             + sum_j c[m, j] L[n, j]
+ * with a(m,k), w(n,k) the dequantized code values (INT4 integers, E4M3 codebook
+ * centroids, or E2M1 x UE4M3 block scale) and one group spanning all of K for
+ * non-INT4 weights.
+ *   a_fmt/w_fmt  (RQ_INT4, RQ_INT4) | (RQ_LM16, RQ_LM16) | (RQ_LM16, RQ_LM4) |
+ *          (RQ_NVFP4, RQ_NVFP4).
+ *   a_codes/w_codes, a_scale/w_scale, a_bscale/w_bscale: as produced above.
+ *   a_lut/w_lut  [host, 16 / 4 bytes] E4M3 value of each codebook index
+ *          (rq_make_codebook's centroids_e4m3) for LM formats; NULL otherwise.
+ *   c, L, r  [device] low-rank branch (r == 32) or NULL / 0.
+ *   Y      [device, M x N] FP32 (out_fp32 = 1) or BF16 (out_fp32 = 0).
+ *   Shapes: M >= 1, N % 32 == 0, K % 128 == 0 (K % 256 == 0 for NVFP4).
+ */
+rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int32_t K, const uint8_t* a_codes,
+                         const float* a_scale, const uint8_t* a_bscale, const uint8_t* w_codes,
+                         const float* w_scale, const uint8_t* w_bscale, const uint8_t* a_lut,
+                         const uint8_t* w_lut, const uint16_t* c, const uint16_t* L, int32_t r, void* Y,
+                         int32_t out_fp32, int32_t* status, void* stream);
+
+/*
+ * rq_read_status -- synchronises `stream`, reads the device status word and
+ * returns RQ_OK, RQ_ERR_TIMEOUT (a kernel gave up a bounded wait; the word is
+ * left set), or RQ_ERR_CUDA.  `code_out` (host, may be NULL) receives the word.
+ */
+rq_status rq_read_status(const int32_t* status, void* stream, int32_t* code_out);
+
+/* Message for the last error returned on the calling thread ("" if none). */
+const char* rq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RQ_H_ */

@@ -1,0 +1,218 @@
+// C ABI of the rotated W4A4 linear layer (declared in include/rq.h): argument
+// checking, host-side table preparation and kernel dispatch.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "../../include/rq.h"
+#include "rq_host.h"
+#include "rq_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+rq_status fail(rq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+rq_status ok() {
+  g_err[0] = 0;
+  return RQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows, int32_t K, int32_t block,
+                          const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r,
+                          const void* coef, const void* codes, const void* scale, const void* bscale) {
+  const bool fmt_ok = fmt == RQ_INT4 || fmt == RQ_LM16 || fmt == RQ_NVFP4 || (weight && fmt == RQ_LM4);
+  if (!fmt_ok) return fail(RQ_ERR_INVALID_ARG, "unknown or unsupported format %d", fmt);
+  if (rows < 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape rows=%d K=%d", rows, K);
+  if (block != 128 && block != 256 && block != 512)
+    return fail(RQ_ERR_UNSUPPORTED, "block %d: the device path supports 128, 256, 512", block);
+  if (K % block) return fail(RQ_ERR_INVALID_ARG, "K=%d is not a multiple of block=%d", K, block);
+  if (K > 16384) return fail(RQ_ERR_UNSUPPORTED, "K=%d exceeds 16384", K);
+  if (K % 128) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of 128", K);
+  if (fmt == RQ_NVFP4 && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs K %% 256 == 0 (K=%d)", K);
+  if (!X || !rot || !codes || !scale) return fail(RQ_ERR_INVALID_ARG, "null input/output pointer");
+  if ((fmt == RQ_LM16 || fmt == RQ_LM4) && !boundaries)
+    return fail(RQ_ERR_INVALID_ARG, "codebook format needs boundaries");
+  if (fmt == RQ_NVFP4 && !bscale) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs block_scale");
+  if (U) {
+    if (r != 32) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r == 32 (got %d)", r);
+    if (!coef) return fail(RQ_ERR_INVALID_ARG, "U given without a coefficient output");
+    if (!aligned16(U) || !aligned16(coef)) return fail(RQ_ERR_ALIGNMENT, "U / coefficient output not 16-byte aligned");
+  }
+  if (!aligned16(X) || !aligned16(rot) || !aligned16(codes) || !aligned16(scale) || (bscale && !aligned16(bscale)))
+    return fail(RQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+  return RQ_OK;
+}
+
+rq_status run_k1(int32_t fmt, bool weight, const uint16_t* X, int32_t rows, int32_t K, int32_t block,
+                 const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r, uint16_t* coef,
+                 uint8_t* codes, float* scale, uint8_t* bscale, int32_t* status, void* stream) {
+  rq_status s = check_rows_call(fmt, weight, X, rows, K, block, rot, boundaries, U, r, coef, codes, scale, bscale);
+  if (s != RQ_OK) return s;
+  if (rows == 0) return ok();
+  rq::K1Launch a{};
+  a.fmt = fmt;
+  a.weight = weight ? 1 : 0;
+  a.x = X;
+  a.rows = rows;
+  a.K = K;
+  a.block = block;
+  a.rot = rot;
+  a.inv_sqrt_b = (float)(1.0 / std::sqrt((double)block));
+  a.sqrtK = std::sqrt((float)K);
+  a.nbnd = fmt == RQ_LM16 ? 15 : fmt == RQ_LM4 ? 3 : 0;
+  a.bnd = boundaries;
+  a.U = U;
+  a.r = U ? r : 0;
+  a.coef = coef;
+  a.codes = codes;
+  a.scale = scale;
+  a.bscale = bscale;
+  a.status = status;
+  a.num_sms = num_sms();
+  cudaError_t e = rq::launch_k1(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "rotate/quantize launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rq_last_error(void) { return g_err; }
+
+rq_status rq_make_rotation(int32_t K, int32_t block, uint64_t seed, int8_t* sign, int32_t* perm, int32_t* rot) {
+  if (K <= 0 || block < 2 || (block & (block - 1)) || K % block)
+    return fail(RQ_ERR_INVALID_ARG, "K=%d must be a positive multiple of a power-of-two block (block=%d)", K, block);
+  rq::make_rotation(K, seed, sign, perm, rot);
+  return ok();
+}
+
+rq_status rq_make_codebook(int32_t K, int32_t levels, double* centroids, double* boundaries, float* boundaries_f32,
+                           uint8_t* centroids_e4m3) {
+  if (K < 4) return fail(RQ_ERR_INVALID_ARG, "K=%d too small", K);
+  if (levels != 4 && levels != 16) return fail(RQ_ERR_UNSUPPORTED, "levels=%d (4 or 16)", levels);
+  std::vector<double> c, b;
+  if (!rq::lloyd_max(K, levels, c, b)) return fail(RQ_ERR_INVALID_ARG, "Lloyd iteration did not converge");
+  for (int i = 0; i < levels; ++i) {
+    if (centroids) centroids[i] = c[i];
+    if (centroids_e4m3) centroids_e4m3[i] = rq::e4m3_encode((double)(float)c[i]);
+  }
+  for (int i = 0; i < levels - 1; ++i) {
+    if (boundaries) boundaries[i] = b[i];
+    if (boundaries_f32) boundaries_f32[i] = (float)b[i];
+  }
+  return ok();
+}
+
+rq_status rq_pca_basis(const uint16_t* calib, int32_t n, int32_t K, int32_t r, uint16_t* U, double* eigenvalues) {
+  if (!calib || !U) return fail(RQ_ERR_INVALID_ARG, "null pointer");
+  if (r < 1 || r > 64 || n < r || K < r) return fail(RQ_ERR_INVALID_ARG, "bad PCA shape n=%d K=%d r=%d", n, K, r);
+  if (!rq::pca_basis(calib, n, K, r, U, eigenvalues))
+    return fail(RQ_ERR_INVALID_ARG, "calibration tokens have rank below r");
+  return ok();
+}
+
+rq_status rq_rotate_quantize_act(int32_t fmt, const uint16_t* X, int32_t M, int32_t K, int32_t block,
+                                 const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r,
+                                 uint16_t* c_out, uint8_t* codes, float* scale, uint8_t* block_scale,
+                                 int32_t* status, void* stream) {
+  return run_k1(fmt, false, X, M, K, block, rot, boundaries, U, r, c_out, codes, scale, block_scale, status, stream);
+}
+
+rq_status rq_quantize_weights(int32_t fmt, const uint16_t* W, int32_t N, int32_t K, int32_t block,
+                              const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r,
+                              uint16_t* L_out, uint8_t* codes, float* scale, uint8_t* block_scale,
+                              int32_t* status, void* stream) {
+  return run_k1(fmt, true, W, N, K, block, rot, boundaries, U, r, L_out, codes, scale, block_scale, status, stream);
+}
+
+rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int32_t K, const uint8_t* a_codes,
+                         const float* a_scale, const uint8_t* a_bscale, const uint8_t* w_codes,
+                         const float* w_scale, const uint8_t* w_bscale, const uint8_t* a_lut,
+                         const uint8_t* w_lut, const uint16_t* c, const uint16_t* L, int32_t r, void* Y,
+                         int32_t out_fp32, int32_t* status, void* stream) {
+  const bool pair_ok = (a_fmt == RQ_INT4 && w_fmt == RQ_INT4) || (a_fmt == RQ_LM16 && w_fmt == RQ_LM16) ||
+                       (a_fmt == RQ_LM16 && w_fmt == RQ_LM4) || (a_fmt == RQ_NVFP4 && w_fmt == RQ_NVFP4);
+  if (!pair_ok) return fail(RQ_ERR_UNSUPPORTED, "format pair (%d, %d) not supported", a_fmt, w_fmt);
+  if (M < 0 || N <= 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape M=%d N=%d K=%d", M, N, K);
+  if (N % 32) return fail(RQ_ERR_INVALID_ARG, "N=%d must be a multiple of 32", N);
+  if (K % 128) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of 128", K);
+  if (a_fmt == RQ_NVFP4 && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs K %% 256 == 0 (K=%d)", K);
+  if (!a_codes || !a_scale || !w_codes || !w_scale || !Y) return fail(RQ_ERR_INVALID_ARG, "null pointer");
+  if (a_fmt == RQ_NVFP4 && (!a_bscale || !w_bscale)) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs block scales");
+  if (a_fmt == RQ_LM16 && (!a_lut || !w_lut)) return fail(RQ_ERR_INVALID_ARG, "codebook formats need LUTs");
+  if ((c != nullptr) != (L != nullptr)) return fail(RQ_ERR_INVALID_ARG, "c and L must both be given or both NULL");
+  if (c && r != 32) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r == 32 (got %d)", r);
+  const void* ptrs[] = {a_codes, a_scale, w_codes, w_scale, Y, a_bscale, w_bscale, c, L};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return fail(RQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+  if (M == 0) return ok();
+  rq::GemmLaunch g{};
+  g.a_fmt = a_fmt;
+  g.w_fmt = w_fmt;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.a_codes = a_codes;
+  g.a_scale = a_scale;
+  g.a_bscale = a_bscale;
+  g.w_codes = w_codes;
+  g.w_scale = w_scale;
+  g.w_bscale = w_bscale;
+  if (a_fmt == RQ_INT4) {
+    for (int i = 0; i < 16; ++i) {
+      const int v = i < 8 ? i : i - 16;  // two's-complement nibble
+      g.a_lut[i] = g.w_lut[i] = rq::e4m3_encode((double)v);
+    }
+  } else if (a_fmt == RQ_LM16) {
+    std::memcpy(g.a_lut, a_lut, 16);
+    std::memcpy(g.w_lut, w_lut, w_fmt == RQ_LM4 ? 4 : 16);
+  }
+  g.c = c;
+  g.L = L;
+  g.r = c ? r : 0;
+  g.Y = Y;
+  g.out_fp32 = out_fp32 ? 1 : 0;
+  g.status = status;
+  g.num_sms = num_sms();
+  const char* why = nullptr;
+  cudaError_t e = rq::launch_gemm(g, static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess)
+    return fail(RQ_ERR_CUDA, "GEMM launch failed: %s%s%s", cudaGetErrorString(e), why ? " / " : "", why ? why : "");
+  return ok();
+}
+
+rq_status rq_read_status(const int32_t* status, void* stream, int32_t* code_out) {
+  if (!status) return fail(RQ_ERR_INVALID_ARG, "null status");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "stream sync failed: %s", cudaGetErrorString(e));
+  int32_t v = 0;
+  e = cudaMemcpy(&v, status, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "status read failed: %s", cudaGetErrorString(e));
+  if (code_out) *code_out = v;
+  if (v != 0) return fail(RQ_ERR_TIMEOUT, "a kernel gave up a bounded wait (code 0x%x)", v);
+  return ok();
+}
+
+}  // extern "C"

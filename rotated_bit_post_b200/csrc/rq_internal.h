@@ -1,0 +1,57 @@
+// Internal launch descriptors shared by the C-ABI layer and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#define RQ_FMT_INT4 1
+#define RQ_FMT_LM16 2
+#define RQ_FMT_NVFP4 3
+#define RQ_FMT_LM4 4
+
+namespace rq {
+
+struct K1Launch {
+  int fmt;
+  int weight;              // 1: weight rows (INT4 per-128-group scales, L = W U)
+  const uint16_t* x;
+  int rows, K, block;
+  const int32_t* rot;
+  float inv_sqrt_b, sqrtK;
+  int nbnd;
+  const float* bnd;        // host, nbnd entries
+  const uint16_t* U;
+  int r;
+  uint16_t* coef;
+  uint8_t* codes;
+  float* scale;
+  uint8_t* bscale;
+  int32_t* status;
+  int num_sms;
+};
+
+cudaError_t launch_k1(const K1Launch& a, cudaStream_t st);
+
+struct GemmLaunch {
+  int a_fmt, w_fmt;
+  int M, N, K;
+  const uint8_t* a_codes;
+  const float* a_scale;
+  const uint8_t* a_bscale;
+  const uint8_t* w_codes;
+  const float* w_scale;
+  const uint8_t* w_bscale;
+  uint8_t a_lut[16];       // e4m3 bytes per code (FP8 path)
+  uint8_t w_lut[16];
+  const uint16_t* c;       // M x r BF16 (low-rank branch) or null
+  const uint16_t* L;       // N x r BF16
+  int r;
+  void* Y;
+  int out_fp32;
+  int32_t* status;
+  int num_sms;
+};
+
+cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why);
+
+}  // namespace rq

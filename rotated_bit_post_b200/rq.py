@@ -1,0 +1,192 @@
+"""Python binding of the C ABI in include/rq.h (argument marshalling only).
+
+Every function keeps the C name.  Device buffers are torch CUDA tensors (their
+data pointers are passed through); host tables are numpy arrays.  All compute
+runs in the CUDA library ``librq.so``; if the library is missing or cannot be
+loaded, every call raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+INT4, LM16, NVFP4, LM4 = 1, 2, 3, 4
+FORMATS = {"int4": INT4, "lm16": LM16, "nvfp4": NVFP4, "lm4": LM4}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librq.so")
+
+_lib = None
+
+_c_i32, _c_u64, _c_p = ctypes.c_int32, ctypes.c_uint64, ctypes.c_void_p
+
+# (name, restype, argtypes) -- mirrors include/rq.h
+SIGNATURES = [
+    ("rq_make_rotation", _c_i32, [_c_i32, _c_i32, _c_u64, _c_p, _c_p, _c_p]),
+    ("rq_make_codebook", _c_i32, [_c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p]),
+    ("rq_pca_basis", _c_i32, [_c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p]),
+    ("rq_rotate_quantize_act", _c_i32,
+     [_c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    ("rq_quantize_weights", _c_i32,
+     [_c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    ("rq_w4a4_linear", _c_i32,
+     [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
+      _c_i32, _c_p, _c_i32, _c_p, _c_p]),
+    ("rq_read_status", _c_i32, [_c_p, _c_p, _c_p]),
+    ("rq_last_error", ctypes.c_char_p, []),
+]
+
+
+class RQError(RuntimeError):
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+def lib():
+    """Load librq.so (raises if it is missing: the library is the only path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run python -m rotated_bit_post_b200.build)")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _check(fn, code):
+    if code != 0:
+        raise RQError(fn, code, lib().rq_last_error().decode())
+
+
+def _np_ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dev(t):
+    """Device pointer of a torch CUDA tensor (or None)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device buffer expected (torch CUDA tensor)")
+    if not t.is_contiguous():
+        raise ValueError("device buffers must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------------ host calls
+def rq_make_rotation(K: int, block: int, seed: int = 0):
+    """-> (sign int8[K], perm int32[K], rot int32[K] signed permutation)."""
+    sign = np.empty(K, np.int8)
+    perm = np.empty(K, np.int32)
+    rot = np.empty(K, np.int32)
+    _check("rq_make_rotation", lib().rq_make_rotation(K, block, seed, _np_ptr(sign), _np_ptr(perm), _np_ptr(rot)))
+    return sign, perm, rot
+
+
+def rq_make_codebook(K: int, levels: int):
+    """-> dict(centroids f64, boundaries f64, boundaries_f32, centroids_e4m3 uint8)."""
+    c = np.empty(levels, np.float64)
+    b = np.empty(levels - 1, np.float64)
+    bf = np.empty(levels - 1, np.float32)
+    e = np.empty(levels, np.uint8)
+    _check("rq_make_codebook", lib().rq_make_codebook(K, levels, _np_ptr(c), _np_ptr(b), _np_ptr(bf), _np_ptr(e)))
+    return {"centroids": c, "boundaries": b, "boundaries_f32": bf, "centroids_e4m3": e}
+
+
+def rq_pca_basis(calib_bf16: np.ndarray, r: int):
+    """calib: uint16 BF16 bits [n, K] -> (U uint16 [K, r], eigenvalues f64 [r])."""
+    calib_bf16 = np.ascontiguousarray(calib_bf16, dtype=np.uint16)
+    n, K = calib_bf16.shape
+    U = np.empty((K, r), np.uint16)
+    ev = np.empty(r, np.float64)
+    _check("rq_pca_basis", lib().rq_pca_basis(_np_ptr(calib_bf16), n, K, r, _np_ptr(U), _np_ptr(ev)))
+    return U, ev
+
+
+# ---------------------------------------------------------------- device calls
+def rq_rotate_quantize_act(fmt, X, block, rot, boundaries, U, c_out, codes, scale, block_scale, status,
+                           stream=None, r=None):
+    M, K = X.shape
+    bnd = None if boundaries is None else np.ascontiguousarray(boundaries, np.float32)
+    rr = (U.shape[1] if U is not None else 0) if r is None else r
+    _check("rq_rotate_quantize_act", lib().rq_rotate_quantize_act(
+        fmt, _dev(X), M, K, block, _dev(rot), _np_ptr(bnd), _dev(U), rr, _dev(c_out), _dev(codes), _dev(scale),
+        _dev(block_scale), _dev(status), _stream(stream)))
+
+
+def rq_quantize_weights(fmt, W, block, rot, boundaries, U, L_out, codes, scale, block_scale, status,
+                        stream=None, r=None):
+    N, K = W.shape
+    bnd = None if boundaries is None else np.ascontiguousarray(boundaries, np.float32)
+    rr = (U.shape[1] if U is not None else 0) if r is None else r
+    _check("rq_quantize_weights", lib().rq_quantize_weights(
+        fmt, _dev(W), N, K, block, _dev(rot), _np_ptr(bnd), _dev(U), rr, _dev(L_out), _dev(codes), _dev(scale),
+        _dev(block_scale), _dev(status), _stream(stream)))
+
+
+def rq_w4a4_linear(a_fmt, w_fmt, M, N, K, a_codes, a_scale, a_bscale, w_codes, w_scale, w_bscale, a_lut, w_lut,
+                   c, L, Y, out_fp32, status, stream=None):
+    al = None if a_lut is None else np.ascontiguousarray(a_lut, np.uint8)
+    wl = None if w_lut is None else np.ascontiguousarray(w_lut, np.uint8)
+    r = 0 if c is None else c.shape[1]
+    _check("rq_w4a4_linear", lib().rq_w4a4_linear(
+        a_fmt, w_fmt, M, N, K, _dev(a_codes), _dev(a_scale), _dev(a_bscale), _dev(w_codes), _dev(w_scale),
+        _dev(w_bscale), _np_ptr(al), _np_ptr(wl), _dev(c), _dev(L), r, _dev(Y), int(out_fp32), _dev(status),
+        _stream(stream)))
+
+
+def rq_read_status(status, stream=None):
+    code = ctypes.c_int32(0)
+    rc = lib().rq_read_status(_dev(status), _stream(stream), ctypes.byref(code))
+    if rc not in (0, 5):
+        _check("rq_read_status", rc)
+    return rc, code.value
+
+
+def rq_last_error() -> str:
+    return lib().rq_last_error().decode()
+
+
+# ------------------------------------------------------- buffer-size helpers
+def sf_bytes(rows: int, K: int) -> int:
+    """Size of an NVFP4 block-scale buffer (128-row x 64-column tiles of 512 B)."""
+    return ((rows + 127) // 128) * (K // 64) * 512
+
+
+def act_buffers(fmt: int, M: int, K: int, r: int = 0, device="cuda"):
+    """Caller-owned output buffers for rq_rotate_quantize_act (torch, uninitialised)."""
+    import torch
+    out = {
+        "codes": torch.empty((M, K // 2), dtype=torch.uint8, device=device),
+        "scale": torch.empty(M, dtype=torch.float32, device=device),
+        "block_scale": torch.zeros(sf_bytes(M, K), dtype=torch.uint8, device=device) if fmt == NVFP4 else None,
+        "c": torch.empty((M, r), dtype=torch.int16, device=device) if r else None,
+    }
+    return out
+
+
+def weight_buffers(fmt: int, N: int, K: int, r: int = 0, device="cuda"):
+    import torch
+    cols = K // 4 if fmt == LM4 else K // 2
+    return {
+        "codes": torch.empty((N, cols), dtype=torch.uint8, device=device),
+        "scale": torch.empty((K // 128, N) if fmt == INT4 else (N,), dtype=torch.float32, device=device),
+        "block_scale": torch.zeros(sf_bytes(N, K), dtype=torch.uint8, device=device) if fmt == NVFP4 else None,
+        "L": torch.empty((N, r), dtype=torch.int16, device=device) if r else None,
+    }
