@@ -9,15 +9,20 @@
 // NVFP4 on Blackwell.)
 //
 // Two mainloops, one epilogue:
-//  * FP8 path (INT4 or Lloyd-Max codes, 4-bit activations, 4- or 2-bit
-//    weights): TMA brings the packed codes into shared memory; four expansion
-//    warps turn every code into its exactly representable E4M3 byte through a
-//    16-entry byte LUT (prmt) and write the 128-byte-swizzled K-major operand
-//    tiles that tcgen05.mma.kind::f8f6f4 reads; one thread issues the MMAs into
-//    a TMEM accumulator.  INT4 weights carry one scale per 128 rotated
-//    coordinates, so every 128-wide K group is accumulated into its own TMEM
-//    partial (double-buffered) and the epilogue folds s_w[g, n] * partial into
-//    a TMEM running sum while the tensor core works on the next group.
+//  * Codebook path (Lloyd-Max codes, 4-bit activations, 4- or 2-bit weights):
+//    TMA brings the packed codes into shared memory; expansion warps turn every
+//    code into its exactly representable E4M3 byte through a 16-entry byte LUT
+//    (prmt) and write the 128-byte-swizzled K-major operand tiles that
+//    tcgen05.mma.kind::f8f6f4 reads; one thread issues the MMAs into TMEM.
+//  * INT4 path: a two's-complement nibble v placed in the high half of a byte
+//    is the int8 value 16 v, so expansion is two masks and a shift per eight
+//    codes (even and odd codes land in separate words; A and B use the same
+//    order, which a dot product over k does not see) and
+//    tcgen05.mma.kind::i8 accumulates 256 * sum(qa qw) exactly in S32.  INT4
+//    weights carry one scale per 128 rotated coordinates, so every 128-wide K
+//    group is accumulated into its own TMEM partial (three buffers) and the
+//    epilogue folds (s_w[g, n] / 256) * partial into running sums held in
+//    registers while the tensor core works on the next groups.
 //  * NVFP4 path: TMA brings packed E2M1 tiles (128B swizzle) and 1-D bulk copies
 //    bring the UE4M3 block scales, already in the 128x4 tile layout K1 writes;
 //    tcgen05.cp moves the scales into TMEM and
@@ -80,6 +85,18 @@ __device__ __forceinline__ uint32_t lut16x4(uint32_t x, const uint32_t (&L)[4]) 
   return prmt(lo, hi, pick);
 }
 
+// Eight 4-bit codes (one 32-bit word, code i in bits 4i..4i+3) -> eight LUT
+// bytes: o0 = codes 0-3, o1 = codes 4-7.  prmt reads only the low 16 bits of
+// its selector, so the high codes are shifted down once.
+__device__ __forceinline__ void lut16x8(uint32_t w, const uint32_t (&L)[4], uint32_t& o0, uint32_t& o1) {
+  const uint32_t sel = w & 0x77777777u;
+  const uint32_t sel_hi = sel >> 16;
+  const uint32_t pick = ((w >> 1) & 0x44444444u) | 0x32103210u;
+  const uint32_t pick_hi = pick >> 16;
+  o0 = prmt(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), pick);
+  o1 = prmt(prmt(L[0], L[1], sel_hi), prmt(L[2], L[3], sel_hi), pick_hi);
+}
+
 // Eight 2-bit codes (bits 0-15 of x) -> eight LUT bytes (lo word: codes 0-3).
 __device__ __forceinline__ void lut4x8(uint32_t x, uint32_t L0, uint32_t& o0, uint32_t& o1) {
   uint32_t t = (x | (x << 8)) & 0x00FF00FFu;
@@ -112,6 +129,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
       "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
       : "memory");
+}
+// 32 lanes x 32 bit, 16 consecutive columns -> 16 registers per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -148,6 +174,10 @@ __device__ __forceinline__ void store_row32(void* Y, int out_fp32, int N, int m,
 __host__ __device__ constexpr uint32_t idesc_f8(int n) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
+// Signed 8-bit A and B (format 1), S32 accumulator (format 2).
+__host__ __device__ constexpr uint32_t idesc_i8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_bf16(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
@@ -157,34 +187,87 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int n) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
+// ===================================================================== shared
+// Named barrier among the epilogue warps.
+template <int NT>
+__device__ __forceinline__ void epi_bar_n() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
+__device__ __forceinline__ void epi_bar() { epi_bar_n<128>(); }
+
+__device__ __forceinline__ void load_scales_smem(float* slot, const float* src, int n0, int N, int BNv, int tid) {
+  for (int i = tid; i < BNv; i += 128) slot[i] = n0 + i < N ? __ldg(src + n0 + i) : 0.f;
+}
+
+// Epilogue of one 32-column chunk for a finished (non-grouped) accumulator:
+// y = acc * (s_a[m] * s_w[n]) (+ low-rank), stored to Y.
+__device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t tacc, uint32_t tlr, bool lr,
+                                                const float* sw, float sa, int row, int nc) {
+  uint32_t acc[32];
+  tmem_ld32(tacc, acc);
+  uint32_t l[32];
+  if (lr) tmem_ld32(tlr, l);
+  tmem_ld_wait();
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const float4 w4 = *reinterpret_cast<const float4*>(sw + i);
+    v[i] = __uint_as_float(acc[i]) * (sa * w4.x);
+    v[i + 1] = __uint_as_float(acc[i + 1]) * (sa * w4.y);
+    v[i + 2] = __uint_as_float(acc[i + 2]) * (sa * w4.z);
+    v[i + 3] = __uint_as_float(acc[i + 3]) * (sa * w4.w);
+  }
+  if (lr) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += __uint_as_float(l[i]);
+  }
+  if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, nc, v);
+}
+
 // ====================================================================== FP8
-// Shared-memory plan (per CTA), all operand buffers 1024-byte aligned:
+// Persistent, warp-specialised.  Shared-memory plan (operand buffers 1024-B aligned):
 //   packed A  [SP][128 x 64 B]   (TMA, 64B swizzle)
 //   packed B  [SP][BN x WROW]    (TMA, 64B swizzle; 32B swizzle for 2-bit codes)
 //   e4m3 A    [SE][128 x 128 B]  (128B swizzle, K-major UMMA operand)
 //   e4m3 B    [SE][BN x 128 B]
-//   c tile    [128 x 64 B], L tile [BN x 64 B] (64B swizzle)
-//   barriers, TMEM base address, abort flag
+//   c / L     [128 x 64 B] / [BN x 64 B] (64B swizzle, BN == 128 only)
+//   weight-scale slots [2][BN] FP32, barriers, TMEM address, abort flag
 template <int BN, int WBITS>
 struct Fp8Plan {
-  static constexpr int SP = 4, SE = 3;
-  static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-K tile
+  static constexpr int SP = BN == 256 ? 3 : 4, SE = BN == 256 ? 3 : 4;
+  static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-wide K tile
   static constexpr int PA = BM * 64, PB = BN * WROW, EA = BM * 128, EB = BN * 128;
+  static constexpr bool LR = BN == 128;
   static constexpr int OFF_PA = 0;
   static constexpr int OFF_PB = OFF_PA + SP * PA;
-  static constexpr int OFF_EA = OFF_PB + SP * PB;
+  static constexpr int OFF_EA = ((OFF_PB + SP * PB) + 1023) & ~1023;
   static constexpr int OFF_EB = OFF_EA + SE * EA;
   static constexpr int OFF_C = OFF_EB + SE * EB;
-  static constexpr int OFF_L = OFF_C + BM * 64;
-  static constexpr int OFF_BAR = OFF_L + BN * 64;
-  static constexpr int NBAR = 2 * SP + 2 * SE + 4 + 2;
+  static constexpr int OFF_L = OFF_C + (LR ? BM * 64 : 0);
+  static constexpr int OFF_SC = OFF_L + (LR ? BN * 64 : 0);
+  static constexpr int SCS = 4;                                // grouped scale ring depth
+  static constexpr int OFF_BAR = OFF_SC + (SCS * BN * 4 > 2 * BN * 4 ? SCS * BN * 4 : 2 * BN * 4);
+  static constexpr int NBAR = 2 * SP + 2 * SE + 6 + 4 + 2 * SCS;
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
 };
 
-// TMEM columns: acc[0] at 0, acc[1] at BN, running sum at 2BN, low-rank at 3BN.
-template <int BN, int WBITS>
-__global__ void __launch_bounds__(384, 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
+// Threads: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, then the
+// epilogue warps (4 warps; 16 when GROUPED: four per TMEM lane quadrant, each
+// owning 32 of the 128 columns and their running sums) and eight code -> e4m3
+// expansion warps.
+// TMEM columns: GROUPED (INT4 weights, BN = 128): three per-group partials at
+// 0, 128, 256 (the running sum lives in the epilogue's registers), low-rank at
+// 384.  Otherwise: accumulators at 0 and BN (double-buffered across tiles),
+// low-rank at 384 when BN == 128.
+template <bool GROUPED>
+constexpr int fp8_threads() { return GROUPED ? 896 : 512; }
+
+template <int BN, int WBITS, bool GROUPED>
+__global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
   using P = Fp8Plan<BN, WBITS>;
+  constexpr int NW = fp8_threads<GROUPED>() / 32;
+  constexpr int NEPI = GROUPED ? 16 : 4;         // epilogue warps
+  constexpr int EXP0 = 4 + NEPI;                 // first expansion warp
+  constexpr int NXT = (NW - EXP0) * 32;          // expansion threads (256)
+  constexpr int NPART = 3;                       // GROUPED partial buffers
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -193,24 +276,34 @@ __global__ void __launch_bounds__(384, 1) gemm_fp8_kernel(const __grid_constant_
   uint64_t* pempty = pfull + P::SP;        // [SP] expansion -> TMA
   uint64_t* efull = pempty + P::SP;        // [SE] expansion -> MMA
   uint64_t* eempty = efull + P::SE;        // [SE] MMA -> expansion
-  uint64_t* accfull = eempty + P::SE;      // [2]  MMA -> epilogue
-  uint64_t* accempty = accfull + 2;        // [2]  epilogue -> MMA
-  uint64_t* lrfull = accempty + 2;         // low-rank tiles landed
-  uint64_t* lrdone = lrfull + 1;           // low-rank MMA done
+  uint64_t* accfull = eempty + P::SE;      // [3]  MMA -> epilogue
+  uint64_t* accempty = accfull + 3;        // [3]  epilogue -> MMA
+  uint64_t* lrfull = accempty + 3;         // c / L tiles landed (TMA -> MMA)
+  uint64_t* lrsmem_empty = lrfull + 1;     // low-rank MMA read them (MMA -> TMA)
+  uint64_t* lrdone = lrsmem_empty + 1;     // low-rank accumulator ready (MMA -> epilogue)
+  uint64_t* lracc_empty = lrdone + 1;      // epilogue read it (epilogue -> MMA)
+  uint64_t* scfull = lracc_empty + 1;      // [SCS] group scales landed (TMA -> epilogue)
+  uint64_t* scempty = scfull + P::SCS;     // [SCS] epilogue used them (epilogue -> TMA)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P::NBAR);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+  float* sc_slots = reinterpret_cast<float*>(smem + P::OFF_SC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
   const int nk = p.K / 128;                // 128-wide K tiles == INT4 groups
-  const bool grouped = p.w_fmt == RQ_FMT_INT4;
+  constexpr bool grouped = GROUPED;
+  const bool lr = P::LR && p.has_lr;
+  const int nN = (p.N + BN - 1) / BN, nM = (p.M + BM - 1) / BM;
+  const int ntiles = nM * nN;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < P::SP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], 4); }
-    for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], 4); mbar_init(&eempty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+    for (int i = 0; i < P::SP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], NW - EXP0); }
+    for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], NW - EXP0); mbar_init(&eempty[i], 1); }
+    for (int i = 0; i < 3; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], NEPI); }
     mbar_init(lrfull, 1);
+    mbar_init(lrsmem_empty, 1);
     mbar_init(lrdone, 1);
+    mbar_init(lracc_empty, NEPI);
+    for (int i = 0; i < P::SCS; ++i) { mbar_init(&scfull[i], 1); mbar_init(&scempty[i], NEPI); }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm.a);
@@ -228,200 +321,299 @@ __global__ void __launch_bounds__(384, 1) gemm_fp8_kernel(const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      if (p.has_lr) {
-        mbar_expect_tx(lrfull, BM * 64 + BN * 64);
-        tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
-        tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
-      }
-      for (int kt = 0; kt < nk; ++kt) {
-        const int s = kt % P::SP;
-        if (kt >= P::SP && !mbar_wait(&pempty[s], ((kt / P::SP) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
-        mbar_expect_tx(&pfull[s], P::PA + P::PB);
-        tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * 64, m0, &pfull[s]);
-        tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0, &pfull[s]);
+      uint32_t kc = 0;
+      int tc = 0;
+      uint32_t sgc = 0;                    // group-scale ring counter (GROUPED)
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
+        const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+        if (lr) {
+          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          mbar_expect_tx(lrfull, BM * 64 + BN * 64);
+          tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
+          tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
+        }
+        for (int kt = 0; kt < nk; ++kt, ++kc) {
+          if constexpr (GROUPED) {
+            // this group's weight scales s_w[kt, n0 .. n0+127] (one contiguous row slice)
+            const int ss = sgc % P::SCS;
+            if (sgc >= P::SCS && !mbar_wait(&scempty[ss], ((sgc / P::SCS) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+            const uint32_t nbytes = (uint32_t)min(128, p.N - n0) * 4;
+            mbar_expect_tx(&scfull[ss], nbytes);
+            bulk_g2s(sc_slots + ss * 128, p.w_scale + (size_t)kt * p.N + n0, nbytes, &scfull[ss]);
+            ++sgc;
+          }
+          const int s = kc % P::SP;
+          if (kc >= P::SP && !mbar_wait(&pempty[s], ((kc / P::SP) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          mbar_expect_tx(&pfull[s], P::PA + P::PB);
+          tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * 64, m0, &pfull[s]);
+          tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0, &pfull[s]);
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      if (p.has_lr) {
-        if (mbar_wait(lrfull, 0, p.status, ST_TIMEOUT_FULL, abort_flag)) {
+      const uint32_t idesc = GROUPED ? idesc_i8(BN) : idesc_f8(BN);
+      uint32_t kc = 0, gc = 0;
+      int tc = 0;
+      bool ok = true;
+      // The low-rank MMA of a tile is issued after its K loop, when the epilogue
+      // has long finished reading the previous tile's low-rank accumulator.
+      auto lowrank = [&](int tcx) -> bool {
+        if (!(mbar_wait(lrfull, tcx & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
+              (tcx == 0 || mbar_wait(lracc_empty, (tcx - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag))))
+          return false;
+        tc_fence_after();
+        const uint32_t ca = sbase + P::OFF_C, la = sbase + P::OFF_L;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          umma_bf16(tmem + 384, smem_desc(ca + kk * 32, 16, 512, 4), smem_desc(la + kk * 32, 16, 512, 4),
+                    idesc_bf16(BN), kk > 0);
+        tc_commit(lrdone);
+        tc_commit(lrsmem_empty);
+        return true;
+      };
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+        const uint32_t ab = tc & 1;
+        if (!grouped && tc >= 2) {
+          ok = mbar_wait(&accempty[ab], ((tc >> 1) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag);
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t ca = sbase + P::OFF_C, la = sbase + P::OFF_L;
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            umma_bf16(tmem + 3 * BN, smem_desc(ca + kk * 32, 16, 512, 4), smem_desc(la + kk * 32, 16, 512, 4),
-                      idesc_bf16(BN), kk > 0);
-          tc_commit(lrdone);
         }
-      }
-      const uint32_t idesc = idesc_f8(BN);
-      int g = 0;  // accumulator group index
-      for (int kt = 0; kt < nk && !*abort_flag; ++kt) {
-        const int s = kt % P::SE;
-        const bool first_of_group = grouped || kt == 0;
-        const int buf = grouped ? (g & 1) : 0;
-        if (first_of_group && grouped && g >= 2) {
-          if (!mbar_wait(&accempty[buf], ((g >> 1) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag)) break;
-        }
-        if (!mbar_wait(&efull[s], (kt / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_f8(tmem + buf * BN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2), idesc,
-                  (first_of_group && kk == 0) ? 0u : 1u);
-        tc_commit(&eempty[s]);
-        if (grouped) {
-          tc_commit(&accfull[buf]);
-          ++g;
-        }
-      }
-      if (!grouped) tc_commit(&accfull[0]);
-    }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp - 4;                  // TMEM lane quadrant
-    const int row = m0 + q * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
-    const int G = grouped ? nk : 1;
-    bool ok = true;
-    for (int g = 0; g < G && ok; ++g) {
-      const int buf = g & 1;
-      ok = mbar_wait(&accfull[buf], (g >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      const bool last = g == G - 1;
-      if (last && p.has_lr) {
-        ok = mbar_wait(lrdone, 0, p.status, ST_TIMEOUT_MMA, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-      }
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int nc = n0 + ch * 32;
-        uint32_t acc[32];
-        tmem_ld32(tmem + lane_off + buf * BN + ch * 32, acc);
-        float run[32];
-        if (grouped && g > 0) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + 2 * BN + ch * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) run[i] = __uint_as_float(r[i]);
-        } else {
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) run[i] = 0.f;
-        }
-        // weight scales for these 32 columns (broadcast loads)
-        const float* sw = grouped ? p.w_scale + (size_t)g * p.N + nc : p.w_scale + nc;
-        float swv[32];
-        if (nc + 32 <= p.N) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 t = __ldg(reinterpret_cast<const float4*>(sw + i));
-            swv[i] = t.x; swv[i + 1] = t.y; swv[i + 2] = t.z; swv[i + 3] = t.w;
+        for (int kt = 0; kt < nk; ++kt, ++kc) {
+          uint32_t buf = ab;
+          if (grouped) {
+            buf = gc % NPART;
+            if (gc >= NPART) {
+              ok = mbar_wait(&accempty[buf], ((gc / NPART) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+            }
           }
-        } else {
+          const int s = kc % P::SE;
+          ok = mbar_wait(&efull[s], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
+          const bool fresh = grouped || kt == 0;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) swv[i] = nc + i < p.N ? __ldg(sw + i) : 0.f;
+          for (int kk = 0; kk < 4; ++kk) {
+            if constexpr (GROUPED)
+              umma_i8(tmem + buf * 128, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
+                      idesc, (fresh && kk == 0) ? 0u : 1u);
+            else
+              umma_f8(tmem + buf * BN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
+                      idesc, (fresh && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&eempty[s]);
+          if (grouped) {
+            tc_commit(&accfull[buf]);
+            ++gc;
+          }
         }
+        if (!ok) break;
+        if (!grouped) tc_commit(&accfull[ab]);
+        if (lr && !(ok = lowrank(tc))) break;
+      }
+    }
+  } else if (warp >= 4 && warp < EXP0) {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 4;
+    const int q = e & 3;                     // TMEM lane quadrant (warp id % 4)
+    const int tid = threadIdx.x - 128;       // 0 .. 32*NEPI-1
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    uint32_t gc = 0;
+    int tc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+      const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+      const int row = m0 + q * 32 + lane;
+      const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
+      if constexpr (GROUPED) {
+        // per 128-wide K group: running[n] += s_w[g, n] * partial_g[m, n], in
+        // registers; this warp owns columns h*32 .. h*32+31 of the tile.  The
+        // 1/256 of the 16 x 16 code scaling is applied once at the end (exact).
+        const int h = e >> 2;
+        float run[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) run[i] = fmaf(swv[i], __uint_as_float(acc[i]), run[i]);
-        if (!last) {
-          tmem_st32(tmem + lane_off + 2 * BN + ch * 32, run);
-        } else {
-          if (p.has_lr) {
-            uint32_t lr[32];
-            tmem_ld32(tmem + lane_off + 3 * BN + ch * 32, lr);
+        for (int i = 0; i < 32; ++i) run[i] = 0.f;
+        for (int g = 0; g < nk; ++g, ++gc) {
+          const uint32_t buf = gc % NPART;
+          const int ss = gc % P::SCS;
+          ok = mbar_wait(&scfull[ss], (gc / P::SCS) & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
+               mbar_wait(&accfull[buf], (gc / NPART) & 1, p.status, ST_TIMEOUT_MMA, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const float* sw = sc_slots + ss * 128 + h * 32;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t acc[16];
+            tmem_ld16(tmem + lane_off + buf * 128 + h * 32 + c * 16, acc);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) run[i] = fmaf(run[i], sa, __uint_as_float(lr[i]));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) run[i] *= sa;
+            for (int i = 0; i < 16; i += 4) {
+              // S32 partials (|x| < 2^21) convert to FP32 exactly
+              const float4 w4 = *reinterpret_cast<const float4*>(sw + c * 16 + i);
+              run[c * 16 + i] = fmaf(w4.x, __int2float_rn((int)acc[i]), run[c * 16 + i]);
+              run[c * 16 + i + 1] = fmaf(w4.y, __int2float_rn((int)acc[i + 1]), run[c * 16 + i + 1]);
+              run[c * 16 + i + 2] = fmaf(w4.z, __int2float_rn((int)acc[i + 2]), run[c * 16 + i + 2]);
+              run[c * 16 + i + 3] = fmaf(w4.w, __int2float_rn((int)acc[i + 3]), run[c * 16 + i + 3]);
+            }
           }
-          if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, nc, run);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&accempty[buf]);   // the tensor core may reuse this partial
+            mbar_arrive(&scempty[ss]);     // the producer may refill this scale slot
+          }
+        }
+        if (!ok) break;
+        const float sa256 = sa * 0.00390625f;
+        if (lr) {
+          ok = mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t l[16];
+            tmem_ld16(tmem + lane_off + 384 + h * 32 + c * 16, l);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) run[c * 16 + i] = fmaf(run[c * 16 + i], sa256, __uint_as_float(l[i]));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(lracc_empty);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) run[i] *= sa256;
+        }
+        if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, n0 + h * 32, run);
+      } else {
+        const uint32_t ab = tc & 1;
+        float* sw = sc_slots + ab * BN;
+        load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid);
+        epi_bar_n<32 * NEPI>();
+        ok = mbar_wait(&accfull[ab], (tc >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag) &&
+             (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 32; ++ch)
+          epi_chunk_final(p, tmem + lane_off + ab * BN + ch * 32, tmem + lane_off + 384 + ch * 32, lr,
+                          sw + ch * 32, sa, row, n0 + ch * 32);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&accempty[ab]);
+          if (lr) mbar_arrive(lracc_empty);
         }
       }
-      if (!last) tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[buf]);
     }
-  } else if (warp >= 8) {
+  } else if (warp >= EXP0) {
     // ------------------------------------------------------------ code -> e4m3 expansion
-    const int t = threadIdx.x - 256;        // 0..127
+    const int t = threadIdx.x - EXP0 * 32;  // 0 .. NXT-1
     uint32_t LA[4], LW[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) { LA[i] = p.a_lut[i]; LW[i] = p.w_lut[i]; }
-    for (int kt = 0; kt < nk; ++kt) {
-      const int sp = kt % P::SP, se = kt % P::SE;
-      if (!mbar_wait(&pfull[sp], (kt / P::SP) & 1, p.status, ST_TIMEOUT_FULL, abort_flag)) break;
-      if (kt >= P::SE && !mbar_wait(&eempty[se], ((kt / P::SE) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
-      const uint32_t pa = sbase + P::OFF_PA + sp * P::PA, pb = sbase + P::OFF_PB + sp * P::PB;
-      const uint32_t ea = sbase + P::OFF_EA + se * P::EA, eb = sbase + P::OFF_EB + se * P::EB;
-      // A: 128 rows x 4 segments of 16 packed bytes (32 codes each)
+    for (int i = 0; i < 4; ++i) {
+      LA[i] = p.a_lut[i];
+      LW[i] = GROUPED ? LA[i] : p.w_lut[i];   // INT4 x INT4 shares one table
+    }
+    uint32_t kc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int kt = 0; kt < nk; ++kt, ++kc) {
+        const int sp = kc % P::SP, se = kc % P::SE;
+        ok = mbar_wait(&pfull[sp], (kc / P::SP) & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
+             (kc < P::SE || mbar_wait(&eempty[se], ((kc / P::SE) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag));
+        if (!ok) break;
+        const uint32_t pa = sbase + P::OFF_PA + sp * P::PA, pb = sbase + P::OFF_PB + sp * P::PB;
+        const uint32_t ea = sbase + P::OFF_EA + se * P::EA, eb = sbase + P::OFF_EB + se * P::EB;
+        if constexpr (GROUPED) {
+          // INT4 codes -> int8 16 v: word j of a 16-byte segment becomes
+          // {even codes << 4, odd codes} (same k order for A and B)
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int idx = it * 128 + t;
-        const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-        const uint4 v = ld_shared_v4(pa + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[8];
+          for (int it = 0; it < 1024 / NXT; ++it) {
+            const int idx0 = it * NXT + t;
+            const bool isb = idx0 >= 512;
+            const int idx = isb ? idx0 - 512 : idx0;
+            const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
+            const uint32_t src = isb ? pb : pa, dst = isb ? eb : ea;
+            const uint4 v = ld_shared_v4(src + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          o[2 * j] = lut16x4(w[j] & 0xFFFFu, LA);
-          o[2 * j + 1] = lut16x4(w[j] >> 16, LA);
+            for (int j = 0; j < 4; ++j) {
+              o[2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
+              o[2 * j + 1] = w[j] & 0xF0F0F0F0u;
+            }
+            const uint32_t rowb = dst + r * 128;
+            st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+            st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&efull[se]);
+            mbar_arrive(&pempty[sp]);
+          }
+          continue;
         }
-        const uint32_t rowb = ea + r * 128;
-        st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
-        st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
-      }
-      if constexpr (WBITS == 4) {
+        // A: 128 rows x 4 segments of 16 packed bytes (32 codes); 8 consecutive
+        // threads take 8 consecutive rows of one segment (conflict-free both ways)
 #pragma unroll
-        for (int it = 0; it < BN / 32; ++it) {
-          const int idx = it * 128 + t;
+        for (int it = 0; it < 512 / NXT; ++it) {
+          const int idx = it * NXT + t;
           const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-          const uint4 v = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+          const uint4 v = ld_shared_v4(pa + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
           uint32_t o[8];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            o[2 * j] = lut16x4(w[j] & 0xFFFFu, LW);
-            o[2 * j + 1] = lut16x4(w[j] >> 16, LW);
-          }
-          const uint32_t rowb = eb + r * 128;
+          for (int j = 0; j < 4; ++j) lut16x8(w[j], LA, o[2 * j], o[2 * j + 1]);
+          const uint32_t rowb = ea + r * 128;
           st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
           st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
         }
-      } else {
-        // 2-bit weights: 32 packed bytes per row = 2 segments of 64 codes
+        if constexpr (WBITS == 4) {
 #pragma unroll
-        for (int it = 0; it < BN / 64; ++it) {
-          const int idx = it * 128 + t;
-          const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
-          const uint4 v = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o[16];
+          for (int it = 0; it < BN * 4 / NXT; ++it) {
+            const int idx = it * NXT + t;
+            const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
+            const uint4 v = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[8];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            lut4x8(w[j] & 0xFFFFu, LW[0], o[4 * j], o[4 * j + 1]);
-            lut4x8(w[j] >> 16, LW[0], o[4 * j + 2], o[4 * j + 3]);
+            for (int j = 0; j < 4; ++j) lut16x8(w[j], LW, o[2 * j], o[2 * j + 1]);
+            const uint32_t rowb = eb + r * 128;
+            st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+            st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
           }
-          const uint32_t rowb = eb + r * 128;
+        } else {
+          // 2-bit weights: 32 packed bytes per row = 2 segments of 64 codes
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            st_shared_v4(rowb + (((4 * seg + c) ^ (r & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          for (int it = 0; it < BN * 2 / NXT; ++it) {
+            const int idx = it * NXT + t;
+            const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
+            const uint4 v = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              lut4x8(w[j] & 0xFFFFu, LW[0], o[4 * j], o[4 * j + 1]);
+              lut4x8(w[j] >> 16, LW[0], o[4 * j + 2], o[4 * j + 3]);
+            }
+            const uint32_t rowb = eb + r * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              st_shared_v4(rowb + (((4 * seg + c) ^ (r & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          }
         }
-      }
-      fence_proxy_async_smem();  // make the generic-proxy writes visible to the tensor core
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&efull[se]);
-        mbar_arrive(&pempty[sp]);
+        fence_proxy_async_smem();  // make the generic-proxy writes visible to the tensor core
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&efull[se]);
+          mbar_arrive(&pempty[sp]);
+        }
       }
     }
   }
@@ -444,15 +636,20 @@ struct Nvf4Plan {
   static constexpr int PA = BM * 128, PB = BN * 128, SA = BM * 16, SB = BN * 16;
   static constexpr int STAGE = PA + PB + SA + SB;
   static constexpr bool LR = BN == 128;   // the low-rank branch runs with BN = 128 only
+  static constexpr int NACC = BN == 256 ? 1 : 2;
   static constexpr int OFF_C = S * STAGE;
   static constexpr int OFF_L = OFF_C + (LR ? BM * 64 : 0);
-  static constexpr int OFF_BAR = OFF_L + (LR ? BN * 64 : 0);
-  static constexpr int NBAR = 2 * S + 2 + 2;
+  static constexpr int OFF_SC = OFF_L + (LR ? BN * 64 : 0);
+  static constexpr int OFF_BAR = OFF_SC + 2 * BN * 4;
+  static constexpr int NBAR = 2 * S + 4 + 4 + 8;
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
 };
 
-// TMEM columns: acc at 0 (BN), low-rank at 128 (only when BN == 128), SFA at
-// 256..271 (4 MMAs x 4 columns), SFB at 272.. (4 MMAs x BN/32 columns).
+// Persistent.  TMEM columns: accumulator(s) at 0 (BN = 256: one; BN = 128: two,
+// at 0 and 128), low-rank at 384 (BN = 128), scale factors in a ring of slots
+// from column 256 (BN = 256: 4 slots of 48 columns; BN = 128: 4 slots of 32),
+// one slot per k-tile in flight, so a k-tile's tcgen05.cp never waits for the
+// previous k-tile's MMAs to finish reading their scales.
 template <int BN>
 __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
   using P = Nvf4Plan<BN>;
@@ -462,22 +659,33 @@ __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = full + P::S;
-  uint64_t* accfull = empty + P::S;
-  uint64_t* lrfull = accfull + 1;
-  uint64_t* lrdone = lrfull + 1;
+  uint64_t* accfull = empty + P::S;        // [2]
+  uint64_t* accempty = accfull + 2;        // [2]
+  uint64_t* lrfull = accempty + 2;
+  uint64_t* lrsmem_empty = lrfull + 1;
+  uint64_t* lrdone = lrsmem_empty + 1;
+  uint64_t* lracc_empty = lrdone + 1;
+  uint64_t* sffull = lracc_empty + 1;      // [4] scale factors in TMEM (copy warp -> MMA)
+  uint64_t* sfempty = sffull + 4;          // [4] MMAs done with a slot (MMA -> copy warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P::NBAR);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+  float* sc_slots = reinterpret_cast<float*>(smem + P::OFF_SC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
   const int nk = p.K / 256;
   const int ktiles64 = p.K / 64;          // scale tiles per 128 rows
+  const bool lr = P::LR && p.has_lr;
+  const int nN = (p.N + BN - 1) / BN, nM = (p.M + BM - 1) / BM;
+  const int ntiles = nM * nN;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < P::S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    mbar_init(accfull, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
     mbar_init(lrfull, 1);
+    mbar_init(lrsmem_empty, 1);
     mbar_init(lrdone, 1);
+    mbar_init(lracc_empty, 4);
+    for (int i = 0; i < 4; ++i) { mbar_init(&sffull[i], 1); mbar_init(&sfempty[i], 1); }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm.a);
@@ -491,93 +699,142 @@ __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_sfa = tmem + 256, t_sfb = tmem + 272;
+  constexpr uint32_t SF_COLS = 16 + 4 * (BN / 32);   // SFA 4 x 4 columns + SFB 4 x BN/32
+  constexpr int SF_SLOTS = 4;
 
   if (warp == 0) {
     if (lane == 0) {
-      if (P::LR && p.has_lr) {
-        mbar_expect_tx(lrfull, BM * 64 + BN * 64);
-        tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
-        tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
-      }
-      const uint8_t* sfa_src = p.a_bscale + (size_t)(m0 / 128) * ktiles64 * 512;
-      // weight scale tiles that exist (the last tile column may cover only 128 rows)
-      const int nb_valid = min(BN / 128, (p.N + 127) / 128 - n0 / 128);
-      for (int kt = 0; kt < nk; ++kt) {
-        const int s = kt % P::S;
-        if (kt >= P::S && !mbar_wait(&empty[s], ((kt / P::S) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
-        uint8_t* st = smem + s * P::STAGE;
-        mbar_expect_tx(&full[s], P::PA + P::PB + P::SA + nb_valid * 2048);
-        tma_load_2d(st, &tm.a, kt * 128, m0, &full[s]);
-        tma_load_2d(st + P::PA, &tm.b, kt * 128, n0, &full[s]);
-        // 4 scale chunks (k tiles of 64) x 512 B, contiguous in the K1 layout
-        bulk_g2s(st + P::PA + P::PB, sfa_src + (size_t)kt * 4 * 512, 2048, &full[s]);
-        for (int nb = 0; nb < nb_valid; ++nb)
-          bulk_g2s(st + P::PA + P::PB + P::SA + nb * 2048,
-                   p.w_bscale + ((size_t)(n0 / 128 + nb) * ktiles64 + (size_t)kt * 4) * 512, 2048, &full[s]);
+      uint32_t kc = 0;
+      int tc = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
+        const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+        if (lr) {
+          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          mbar_expect_tx(lrfull, BM * 64 + BN * 64);
+          tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
+          tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
+        }
+        const uint8_t* sfa_src = p.a_bscale + (size_t)(m0 / 128) * ktiles64 * 512;
+        // weight scale tiles that exist (the last tile column may cover only 128 rows)
+        const int nb_valid = min(BN / 128, (p.N + 127) / 128 - n0 / 128);
+        for (int kt = 0; kt < nk; ++kt, ++kc) {
+          const int s = kc % P::S;
+          if (kc >= P::S && !mbar_wait(&empty[s], ((kc / P::S) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          uint8_t* st = smem + s * P::STAGE;
+          mbar_expect_tx(&full[s], P::PA + P::PB + P::SA + nb_valid * 2048);
+          tma_load_2d(st, &tm.a, kt * 128, m0, &full[s]);
+          tma_load_2d(st + P::PA, &tm.b, kt * 128, n0, &full[s]);
+          // 4 scale chunks (k tiles of 64) x 512 B, contiguous in the K1 layout
+          bulk_g2s(st + P::PA + P::PB, sfa_src + (size_t)kt * 4 * 512, 2048, &full[s]);
+          for (int nb = 0; nb < nb_valid; ++nb)
+            bulk_g2s(st + P::PA + P::PB + P::SA + nb * 2048,
+                     p.w_bscale + ((size_t)(n0 / 128 + nb) * ktiles64 + (size_t)kt * 4) * 512, 2048, &full[s]);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      if (p.has_lr) {
-        if (mbar_wait(lrfull, 0, p.status, ST_TIMEOUT_FULL, abort_flag)) {
+      const uint32_t idesc = idesc_nvf4(BN);
+      uint32_t kc = 0;
+      int tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+        const uint32_t ab = tc % P::NACC;
+        if (tc >= P::NACC) {
+          ok = mbar_wait(&accempty[ab], ((tc / P::NACC) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        for (int kt = 0; kt < nk; ++kt, ++kc) {
+          const int s = kc % P::S;
+          const int sl = kc % SF_SLOTS;
+          ok = mbar_wait(&full[s], (kc / P::S) & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
+               mbar_wait(&sffull[sl], (kc / SF_SLOTS) & 1, p.status, ST_TIMEOUT_FULL, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t st = sbase + s * P::STAGE;
+          const uint32_t t_sfa = tmem + 256 + sl * SF_COLS, t_sfb = t_sfa + 16;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_nvf4(tmem + ab * BN, smem_desc(st + kk * 32, 16, 1024, 2), smem_desc(st + P::PA + kk * 32, 16, 1024, 2),
+                      idesc, t_sfa + kk * 4, t_sfb + kk * (BN / 32), (kt > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
+          tc_commit(&sfempty[sl]);
+        }
+        if (!ok) break;
+        tc_commit(&accfull[ab]);
+        if (lr) {
+          // low-rank MMA after the K loop (see the codebook kernel)
+          ok = mbar_wait(lrfull, tc & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
+               (tc == 0 || mbar_wait(lracc_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag));
+          if (!ok) break;
           tc_fence_after();
           const uint32_t ca = sbase + P::OFF_C, la = sbase + P::OFF_L;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            umma_bf16(tmem + BN, smem_desc(ca + kk * 32, 16, 512, 4), smem_desc(la + kk * 32, 16, 512, 4),
+            umma_bf16(tmem + 384, smem_desc(ca + kk * 32, 16, 512, 4), smem_desc(la + kk * 32, 16, 512, 4),
                       idesc_bf16(BN), kk > 0);
           tc_commit(lrdone);
+          tc_commit(lrsmem_empty);
         }
       }
-      const uint32_t idesc = idesc_nvf4(BN);
-      for (int kt = 0; kt < nk; ++kt) {
-        const int s = kt % P::S;
-        if (!mbar_wait(&full[s], (kt / P::S) & 1, p.status, ST_TIMEOUT_FULL, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t st = sbase + s * P::STAGE;
-        const uint32_t sfa = st + P::PA + P::PB, sfb = sfa + P::SA;
-        // scale factors -> TMEM: per MMA (K = 64) one 512 B chunk per 128 rows
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale factors -> TMEM
+    // (UE4M3, per MMA one 512 B chunk per 128 rows) into a ring of SF_SLOTS
+    // column groups, on their own issue stream so the copies overlap the MMAs
+    if (lane == 0) {
+      uint32_t kc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        for (int kt = 0; kt < nk; ++kt, ++kc) {
+          const int s = kc % P::S;
+          const int sl = kc % SF_SLOTS;
+          ok = (kc < (uint32_t)SF_SLOTS ||
+                mbar_wait(&sfempty[sl], ((kc / SF_SLOTS) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) &&
+               mbar_wait(&full[s], (kc / P::S) & 1, p.status, ST_TIMEOUT_FULL, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sfa = sbase + s * P::STAGE + P::PA + P::PB, sfb = sfa + P::SA;
+          const uint32_t t_a = tmem + 256 + sl * SF_COLS, t_b = t_a + 16;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          tc_cp_32x128b_warpx4(t_sfa + kk * 4, smem_desc(sfa + kk * 512, 16, 128, 0));
+          for (int kk = 0; kk < 4; ++kk) {
+            tc_cp_32x128b_warpx4(t_a + kk * 4, smem_desc(sfa + kk * 512, 16, 128, 0));
 #pragma unroll
-          for (int nb = 0; nb < BN / 128; ++nb)
-            tc_cp_32x128b_warpx4(t_sfb + kk * (BN / 32) + nb * 4, smem_desc(sfb + nb * 2048 + kk * 512, 16, 128, 0));
+            for (int nb = 0; nb < BN / 128; ++nb)
+              tc_cp_32x128b_warpx4(t_b + kk * (BN / 32) + nb * 4, smem_desc(sfb + nb * 2048 + kk * 512, 16, 128, 0));
+          }
+          tc_commit(&sffull[sl]);
         }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_nvf4(tmem, smem_desc(st + kk * 32, 16, 1024, 2), smem_desc(st + P::PA + kk * 32, 16, 1024, 2), idesc,
-                    t_sfa + kk * 4, t_sfb + kk * (BN / 32), (kt > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&empty[s]);
       }
-      tc_commit(accfull);
     }
   } else if (warp >= 4) {
     const int q = warp - 4;
-    const int row = m0 + q * 32 + lane;
+    const int tid = threadIdx.x - 128;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
-    bool ok = mbar_wait(accfull, 0, p.status, ST_TIMEOUT_MMA, abort_flag);
-    if (ok && p.has_lr) ok = mbar_wait(lrdone, 0, p.status, ST_TIMEOUT_MMA, abort_flag);
-    if (ok) {
+    int tc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+      const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+      const int row = m0 + q * 32 + lane;
+      const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
+      const uint32_t ab = tc % P::NACC;
+      float* sw = sc_slots + (tc & 1) * BN;
+      load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid);
+      epi_bar();
+      ok = mbar_wait(&accfull[ab], (tc / P::NACC) & 1, p.status, ST_TIMEOUT_MMA, abort_flag) &&
+           (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag));
+      if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int nc = n0 + ch * 32;
-        uint32_t acc[32];
-        tmem_ld32(tmem + lane_off + ch * 32, acc);
-        uint32_t lr[32];
-        if (p.has_lr) tmem_ld32(tmem + lane_off + BN + ch * 32, lr);
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float swv = nc + i < p.N ? __ldg(p.w_scale + nc + i) : 0.f;
-          v[i] = __uint_as_float(acc[i]) * (sa * swv);
-          if (p.has_lr) v[i] += __uint_as_float(lr[i]);
-        }
-        if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, nc, v);
+      for (int ch = 0; ch < BN / 32; ++ch)
+        epi_chunk_final(p, tmem + lane_off + ab * BN + ch * 32, tmem + lane_off + 384 + ch * 32, lr, sw + ch * 32,
+                        sa, row, n0 + ch * 32);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&accempty[ab]);
+        if (lr) mbar_arrive(lracc_empty);
       }
     }
   }
@@ -642,7 +899,9 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   gp.Y = a.Y; gp.out_fp32 = a.out_fp32; gp.status = a.status;
 
   const bool nvf4 = a.a_fmt == RQ_FMT_NVFP4;
-  const int BN = (nvf4 && !gp.has_lr) ? 256 : 128;
+  const bool grouped = a.w_fmt == RQ_FMT_INT4;
+  // 128 x 256 tiles unless the INT4 group epilogue or the low-rank branch needs the TMEM
+  const int BN = (grouped || gp.has_lr) ? 128 : 256;
   bool ok = true;
   if (gp.has_lr) {
     ok &= make_map_2d(&tm.c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.c, a.r, a.M, (uint64_t)a.r * 2, 32, BM,
@@ -650,7 +909,9 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     ok &= make_map_2d(&tm.l, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L, a.r, a.N, (uint64_t)a.r * 2, 32, BN,
                       CU_TENSOR_MAP_SWIZZLE_64B);
   }
-  dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM);
+  const int ntiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const int sms = a.num_sms > 0 ? a.num_sms : 148;
+  dim3 grid(ntiles < sms ? ntiles : sms);
   if (nvf4) {
     ok &= make_map_2d(&tm.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, a.K / 2, a.M, a.K / 2, 128, BM,
                       CU_TENSOR_MAP_SWIZZLE_128B);
@@ -670,8 +931,13 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 2, a.N, a.K / 2, 64, BN,
                       CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) { *why = "cuTensorMapEncodeTiled failed"; return cudaErrorInvalidValue; }
-  if (w2) return launch(gemm_fp8_kernel<128, 2>, Fp8Plan<128, 2>::BYTES, grid, 384, tm, gp, st);
-  return launch(gemm_fp8_kernel<128, 4>, Fp8Plan<128, 4>::BYTES, grid, 384, tm, gp, st);
+  if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, 896, tm, gp, st);
+  if (BN == 256) {
+    if (w2) return launch(gemm_fp8_kernel<256, 2, false>, Fp8Plan<256, 2>::BYTES, grid, 512, tm, gp, st);
+    return launch(gemm_fp8_kernel<256, 4, false>, Fp8Plan<256, 4>::BYTES, grid, 512, tm, gp, st);
+  }
+  if (w2) return launch(gemm_fp8_kernel<128, 2, false>, Fp8Plan<128, 2>::BYTES, grid, 512, tm, gp, st);
+  return launch(gemm_fp8_kernel<128, 4, false>, Fp8Plan<128, 4>::BYTES, grid, 512, tm, gp, st);
 }
 
 }  // namespace rq
