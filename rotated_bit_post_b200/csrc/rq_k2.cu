@@ -139,6 +139,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+// run += w * (as_float(x + 0x4B400000) - 1.5 * 2^23) on two lanes of packed
+// FP32 arithmetic.  For |x| < 2^22 the integer add lands x in the mantissa of
+// a float whose unit in the last place is 1, so the subtraction recovers x
+// exactly: an exact S32 -> F32 conversion on the full-rate pipes.
+__device__ __forceinline__ void fma_s32x2(float& r0, float& r1, float w0, float w1, uint32_t x0, uint32_t x1) {
+  asm("{\n\t.reg .b64 f, m, w, r;\n\t"
+      "mov.b64 f, {%2, %3};\n\t"
+      "mov.b64 m, {%6, %6};\n\t"
+      "mov.b64 w, {%4, %5};\n\t"
+      "mov.b64 r, {%0, %1};\n\t"
+      "sub.rn.f32x2 f, f, m;\n\t"
+      "fma.rn.f32x2 r, w, f, r;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "+f"(r0), "+f"(r1)
+      : "r"(x0 + 0x4B400000u), "r"(x1 + 0x4B400000u), "f"(w0), "f"(w1), "f"(12582912.0f));
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Store 32 consecutive outputs of one row (FP32 or BF16), masked to n < N.
@@ -149,7 +165,9 @@ __device__ __forceinline__ void store_row32(void* Y, int out_fp32, int N, int m,
 #pragma unroll
       for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
     } else {
-      for (int i = 0; i < 32 && n0 + i < N; ++i) dst[i] = v[i];
+#pragma unroll
+      for (int i = 0; i < 32; ++i)   // unrolled with predicates: v stays in registers
+        if (n0 + i < N) dst[i] = v[i];
     }
   } else {
     __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(Y) + (size_t)m * N + n0;
@@ -164,7 +182,9 @@ __device__ __forceinline__ void store_row32(void* Y, int out_fp32, int N, int m,
       for (int i = 0; i < 16; i += 4)
         *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
     } else {
-      for (int i = 0; i < 32 && n0 + i < N; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < N) dst[i] = __float2bfloat16_rn(v[i]);
     }
   }
 }
@@ -243,22 +263,25 @@ struct Fp8Plan {
   static constexpr int OFF_C = OFF_EB + SE * EB;
   static constexpr int OFF_L = OFF_C + (LR ? BM * 64 : 0);
   static constexpr int OFF_SC = OFF_L + (LR ? BN * 64 : 0);
-  static constexpr int SCS = 4;                                // grouped scale ring depth
+  static constexpr int SCS = BN == 128 ? 12 : 4;               // grouped scale ring depth (BN 128 only)
   static constexpr int OFF_BAR = OFF_SC + (SCS * BN * 4 > 2 * BN * 4 ? SCS * BN * 4 : 2 * BN * 4);
   static constexpr int NBAR = 2 * SP + 2 * SE + 6 + 4 + 2 * SCS;
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
+  static_assert(BYTES <= 232448, "shared memory plan exceeds 227 KB");
 };
 
 // Threads: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, then the
-// epilogue warps (4 warps; 16 when GROUPED: four per TMEM lane quadrant, each
-// owning 32 of the 128 columns and their running sums) and eight code -> e4m3
-// expansion warps.
+// epilogue warps from warp 4 (4 warps; 16 when GROUPED: four per TMEM lane
+// quadrant, each owning 32 of the 128 columns and their running sums) and the
+// code expansion warps: eight after the epilogue, or, when GROUPED, warps 2-3
+// plus two after the epilogue (704 threads, so that the 16 epilogue warps keep
+// their running sums in registers without spilling).
 // TMEM columns: GROUPED (INT4 weights, BN = 128): three per-group partials at
 // 0, 128, 256 (the running sum lives in the epilogue's registers), low-rank at
 // 384.  Otherwise: accumulators at 0 and BN (double-buffered across tiles),
 // low-rank at 384 when BN == 128.
 template <bool GROUPED>
-constexpr int fp8_threads() { return GROUPED ? 896 : 512; }
+constexpr int fp8_threads() { return GROUPED ? 704 : 512; }
 
 template <int BN, int WBITS, bool GROUPED>
 __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
@@ -266,7 +289,8 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
   constexpr int NW = fp8_threads<GROUPED>() / 32;
   constexpr int NEPI = GROUPED ? 16 : 4;         // epilogue warps
   constexpr int EXP0 = 4 + NEPI;                 // first expansion warp
-  constexpr int NXT = (NW - EXP0) * 32;          // expansion threads (256)
+  constexpr int NXW = GROUPED ? 4 : NW - EXP0;   // expansion warps
+  constexpr int NXT = NXW * 32;                  // expansion threads
   constexpr int NPART = 3;                       // GROUPED partial buffers
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -296,8 +320,8 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
   const int ntiles = nM * nN;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < P::SP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], NW - EXP0); }
-    for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], NW - EXP0); mbar_init(&eempty[i], 1); }
+    for (int i = 0; i < P::SP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], NXW); }
+    for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], NXW); mbar_init(&eempty[i], 1); }
     for (int i = 0; i < 3; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], NEPI); }
     mbar_init(lrfull, 1);
     mbar_init(lrsmem_empty, 1);
@@ -326,12 +350,6 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
       uint32_t sgc = 0;                    // group-scale ring counter (GROUPED)
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
         const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
-        if (lr) {
-          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
-          mbar_expect_tx(lrfull, BM * 64 + BN * 64);
-          tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
-          tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
-        }
         for (int kt = 0; kt < nk; ++kt, ++kc) {
           if constexpr (GROUPED) {
             // this group's weight scales s_w[kt, n0 .. n0+127] (one contiguous row slice)
@@ -347,6 +365,14 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
           mbar_expect_tx(&pfull[s], P::PA + P::PB);
           tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * 64, m0, &pfull[s]);
           tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0, &pfull[s]);
+        }
+        // the tile's low-rank operands go after its K tiles, so waiting for the
+        // previous tile's low-rank MMA never stalls the K-tile prefetch
+        if (lr) {
+          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          mbar_expect_tx(lrfull, BM * 64 + BN * 64);
+          tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
+          tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
         }
       }
     }
@@ -452,12 +478,10 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; i += 4) {
-              // S32 partials (|x| < 2^21) convert to FP32 exactly
+              // S32 partials (|x| <= 256 * 49 * 128 < 2^21) convert to FP32 exactly
               const float4 w4 = *reinterpret_cast<const float4*>(sw + c * 16 + i);
-              run[c * 16 + i] = fmaf(w4.x, __int2float_rn((int)acc[i]), run[c * 16 + i]);
-              run[c * 16 + i + 1] = fmaf(w4.y, __int2float_rn((int)acc[i + 1]), run[c * 16 + i + 1]);
-              run[c * 16 + i + 2] = fmaf(w4.z, __int2float_rn((int)acc[i + 2]), run[c * 16 + i + 2]);
-              run[c * 16 + i + 3] = fmaf(w4.w, __int2float_rn((int)acc[i + 3]), run[c * 16 + i + 3]);
+              fma_s32x2(run[c * 16 + i], run[c * 16 + i + 1], w4.x, w4.y, acc[i], acc[i + 1]);
+              fma_s32x2(run[c * 16 + i + 2], run[c * 16 + i + 3], w4.z, w4.w, acc[i + 2], acc[i + 3]);
             }
           }
           tc_fence_before();
@@ -510,9 +534,9 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
         }
       }
     }
-  } else if (warp >= EXP0) {
-    // ------------------------------------------------------------ code -> e4m3 expansion
-    const int t = threadIdx.x - EXP0 * 32;  // 0 .. NXT-1
+  } else if (warp >= EXP0 || (GROUPED && warp >= 2)) {
+    // ------------------------------------------------------------ code expansion
+    const int t = (GROUPED && warp < 4 ? warp - 2 + (NW - EXP0) : warp - EXP0) * 32 + lane;  // 0 .. NXT-1
     uint32_t LA[4], LW[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -643,6 +667,7 @@ struct Nvf4Plan {
   static constexpr int OFF_BAR = OFF_SC + 2 * BN * 4;
   static constexpr int NBAR = 2 * S + 4 + 4 + 8;
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static_assert(BYTES <= 232448, "shared memory plan exceeds 227 KB");
 };
 
 // Persistent.  TMEM columns: accumulator(s) at 0 (BN = 256: one; BN = 128: two,
@@ -708,12 +733,6 @@ __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant
       int tc = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
         const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
-        if (lr) {
-          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
-          mbar_expect_tx(lrfull, BM * 64 + BN * 64);
-          tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
-          tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
-        }
         const uint8_t* sfa_src = p.a_bscale + (size_t)(m0 / 128) * ktiles64 * 512;
         // weight scale tiles that exist (the last tile column may cover only 128 rows)
         const int nb_valid = min(BN / 128, (p.N + 127) / 128 - n0 / 128);
@@ -729,6 +748,12 @@ __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant
           for (int nb = 0; nb < nb_valid; ++nb)
             bulk_g2s(st + P::PA + P::PB + P::SA + nb * 2048,
                      p.w_bscale + ((size_t)(n0 / 128 + nb) * ktiles64 + (size_t)kt * 4) * 512, 2048, &full[s]);
+        }
+        if (lr) {   // after the K tiles (see the codebook kernel)
+          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          mbar_expect_tx(lrfull, BM * 64 + BN * 64);
+          tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
+          tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
         }
       }
     }
@@ -931,7 +956,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 2, a.N, a.K / 2, 64, BN,
                       CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) { *why = "cuTensorMapEncodeTiled failed"; return cudaErrorInvalidValue; }
-  if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, 896, tm, gp, st);
+  if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<true>(), tm, gp, st);
   if (BN == 256) {
     if (w2) return launch(gemm_fp8_kernel<256, 2, false>, Fp8Plan<256, 2>::BYTES, grid, 512, tm, gp, st);
     return launch(gemm_fp8_kernel<256, 4, false>, Fp8Plan<256, 4>::BYTES, grid, 512, tm, gp, st);
