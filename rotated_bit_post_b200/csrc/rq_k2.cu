@@ -556,24 +556,38 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
         if constexpr (GROUPED) {
           // INT4 codes -> int8 16 v: word j of a 16-byte segment becomes
           // {even codes << 4, odd codes} (same k order for A and B)
+          // loads in batches of four: the shared-memory accesses are ordered,
+          // so batching keeps four in flight at once
+          constexpr int NIT = 1024 / NXT, NB = 4;
 #pragma unroll
-          for (int it = 0; it < 1024 / NXT; ++it) {
-            const int idx0 = it * NXT + t;
-            const bool isb = idx0 >= 512;
-            const int idx = isb ? idx0 - 512 : idx0;
-            const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-            const uint32_t src = isb ? pb : pa, dst = isb ? eb : ea;
-            const uint4 v = ld_shared_v4(src + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o[8];
+          for (int b0 = 0; b0 < NIT; b0 += NB) {
+            uint4 vin[NB];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              o[2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
-              o[2 * j + 1] = w[j] & 0xF0F0F0F0u;
+            for (int j = 0; j < NB; ++j) {
+              const int idx0 = (b0 + j) * NXT + t;
+              const bool isb = idx0 >= 512;
+              const int idx = isb ? idx0 - 512 : idx0;
+              const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
+              vin[j] = ld_shared_v4((isb ? pb : pa) + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
             }
-            const uint32_t rowb = dst + r * 128;
-            st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
-            st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+#pragma unroll
+            for (int j = 0; j < NB; ++j) {
+              const int idx0 = (b0 + j) * NXT + t;
+              const bool isb = idx0 >= 512;
+              const int idx = isb ? idx0 - 512 : idx0;
+              const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
+              const uint32_t dst = isb ? eb : ea;
+              const uint32_t w[4] = {vin[j].x, vin[j].y, vin[j].z, vin[j].w};
+              uint32_t o[8];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                o[2 * q] = (w[q] << 4) & 0xF0F0F0F0u;
+                o[2 * q + 1] = w[q] & 0xF0F0F0F0u;
+              }
+              const uint32_t rowb = dst + r * 128;
+              st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+              st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -585,11 +599,18 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
         }
         // A: 128 rows x 4 segments of 16 packed bytes (32 codes); 8 consecutive
         // threads take 8 consecutive rows of one segment (conflict-free both ways)
+        uint4 va[512 / NXT];
 #pragma unroll
         for (int it = 0; it < 512 / NXT; ++it) {
           const int idx = it * NXT + t;
           const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-          const uint4 v = ld_shared_v4(pa + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+          va[it] = ld_shared_v4(pa + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+        }
+#pragma unroll
+        for (int it = 0; it < 512 / NXT; ++it) {
+          const int idx = it * NXT + t;
+          const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
+          const uint4 v = va[it];
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
           uint32_t o[8];
 #pragma unroll
@@ -599,11 +620,18 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
           st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
         }
         if constexpr (WBITS == 4) {
+          uint4 vb[BN * 4 / NXT];
 #pragma unroll
           for (int it = 0; it < BN * 4 / NXT; ++it) {
             const int idx = it * NXT + t;
             const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-            const uint4 v = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+            vb[it] = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+          }
+#pragma unroll
+          for (int it = 0; it < BN * 4 / NXT; ++it) {
+            const int idx = it * NXT + t;
+            const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
+            const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             uint32_t o[8];
 #pragma unroll
@@ -614,11 +642,18 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
           }
         } else {
           // 2-bit weights: 32 packed bytes per row = 2 segments of 64 codes
+          uint4 vb[BN * 2 / NXT];
 #pragma unroll
           for (int it = 0; it < BN * 2 / NXT; ++it) {
             const int idx = it * NXT + t;
             const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
-            const uint4 v = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
+            vb[it] = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
+          }
+#pragma unroll
+          for (int it = 0; it < BN * 2 / NXT; ++it) {
+            const int idx = it * NXT + t;
+            const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
+            const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             uint32_t o[16];
 #pragma unroll
