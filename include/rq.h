@@ -120,7 +120,8 @@ rq_status rq_pca_basis(const uint16_t* calib, int32_t n, int32_t K, int32_t r, u
  *          K % 128 == 0 (INT4 / LM16), K % 256 == 0 (NVFP4).
  *   rot    [device, K] signed permutation from rq_make_rotation.
  *   boundaries [host, levels-1] FP32 codebook boundaries (RQ_LM16), else NULL.
- *   U, r   [device, K x r] BF16 PCA basis and its rank (r == 32), or NULL / 0.
+ *   U, r   [device, K x r] BF16 PCA basis and its rank (r == 32, K <= 3072:
+ *          U^T is staged whole in shared memory), or NULL / 0.
  *          With U: c = bf16(x U) (FP32, sequential over k) is written to c_out
  *          and the residual x - c U^T is what gets rotated and quantized.
  *   c_out  [device, M x r] BF16 or NULL.
@@ -146,7 +147,8 @@ rq_status rq_rotate_quantize_act(int32_t fmt, const uint16_t* X, int32_t M, int3
  *   fmt    RQ_INT4 (one scale per 128 rotated coordinates) | RQ_LM16 | RQ_LM4 |
  *          RQ_NVFP4.
  *   W      [device, N x K] BF16.
- *   U, r, L_out  optional: L = bf16(W U) [device, N x r] for the low-rank branch
+ *   U, r, L_out  optional (r == 32, K <= 3072): L = bf16(W U) [device, N x r]
+ *          (FP32, sequential over k) for the low-rank branch
  *          (the full row is still what gets quantized).
  *   codes  [device, N x K/2] (RQ_LM4: N x K/4).
  *   scale  [device] RQ_INT4: [K/128][N] group-major; otherwise [N].

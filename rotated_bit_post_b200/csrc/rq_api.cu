@@ -56,6 +56,7 @@ rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows,
   if (fmt == RQ_NVFP4 && !bscale) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs block_scale");
   if (U) {
     if (r != 32) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r == 32 (got %d)", r);
+    if (K > 3072) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports K <= 3072 (got %d)", K);
     if (!coef) return fail(RQ_ERR_INVALID_ARG, "U given without a coefficient output");
     if (!aligned16(U) || !aligned16(coef)) return fail(RQ_ERR_ALIGNMENT, "U / coefficient output not 16-byte aligned");
   }

@@ -8,8 +8,10 @@
 // quantizers (OrbitQuant abstract; TR-DQ Eq. 9).
 //
 // Data flow per CTA (persistent over groups of R rows):
-//   HBM --cp.async.bulk--> smem row buffer (double-buffered, mbarrier)
-//   [projection: c = bf16(x U) sequentially over k, x_res = x - c U^T]
+//   HBM --cp.async.bulk--> smem row buffer (mbarrier)
+//   [projection: c = bf16(x U), each of the R x 32 sums a sequential FP32 chain
+//    over k (one chain per thread, every warp busy); then, in sub-groups of Rs
+//    rows, x_res = x - c U^T (sequential over j) into an FP32 buffer]
 //   a group of L = b/32 lanes owns one b-wide Hadamard block of one row: lane j
 //   of the group holds the 32 consecutive rotated coordinates 32j .. 32j+31,
 //   gathered from smem through the signed-permutation table; butterfly stages
@@ -21,7 +23,9 @@
 // FP32 contract (bit-exact against the CPU oracle): every add/multiply/divide is
 // an explicit round-to-nearest-even intrinsic (no contraction); the only fused
 // multiply-adds are the projection's, whose products of two BF16 values are
-// exact in FP32 so the fused and unfused results agree.
+// exact in FP32 so the fused and unfused results agree.  They are issued as
+// fma.rn.f32.bf16 (BF16 operands, FP32 addend and result), which is the same
+// single rounding of the exact product plus the addend.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -48,7 +52,8 @@ struct __align__(16) K1Params {
   uint8_t* bscale;         // NVFP4 block scales, 128x4 swizzled tiles
   int32_t* status;
   int32_t rows, K, r;
-  int32_t R;               // rows per group
+  int32_t R;               // rows per group (one load)
+  int32_t Rs;              // rows per sub-group (rotation / quantization pass)
   int32_t ngroups;
   float inv_sqrt_b;        // fp32(1/sqrt(block))
   float sqrtK;             // fp32(sqrt(K))
@@ -64,14 +69,34 @@ __device__ __forceinline__ size_t sf_offset(int m, int kb, int K) {
   return ((size_t)(m >> 7) * tiles_k + (kb >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (kb & 3);
 }
 
+// acc + a * b for BF16 a, b (half AH of word a, half BH of word b; 0 = low
+// 16 bits), FP32 acc, one rounding: the product of two BF16 values is exact.
+template <int AH, int BH>
+__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float acc) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, a%4, b%5, %3;\n\t}"
+      : "=f"(d)
+      : "r"(a), "r"(b), "f"(acc), "n"(AH), "n"(BH));
+  return d;
+}
+
+// Projection layout in shared memory: U^T as BF16 rows of KP = K + 8 entries
+// (the 16-byte pad spreads the 32 rows over all banks).
+__host__ __device__ constexpr int ut_pitch(int K) { return K + 8; }
+
 template <int L, int FMT, bool PROJ, bool WEIGHT, int IPW>
 __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quantize(const __grid_constant__ K1Params p) {
   constexpr int B = L * 32;                // Hadamard block
   constexpr int GPW = 32 / L;              // lane groups (block slots) per warp
   constexpr int SLOTS = K1_WARPS * GPW;    // block slots per CTA pass
+  constexpr bool RESID = PROJ && !WEIGHT;  // activations: rotate the residual
+  constexpr int NB = PROJ ? 1 : 2;         // row buffers (prefetch without projection)
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = p.K;
-  const int R = p.R;
+  const int R = p.R, Rs = p.Rs;
   const int nblk = K / B;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -80,30 +105,32 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
   // shuffles stay inside the lane group (groups of one warp may take different branches)
   const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
 
-  // smem layout: [2][R][K] bf16 row buffers | (PROJ) [R][K] fp32 x / residual |
-  // (PROJ) [R][32] fp32 coefficients | (PROJ) [K/2][32] U as BF16 pairs over k |
-  // [R][nblk] fp32 block sum-of-squares | [R][ngrp] u32 amax bits |
-  // [R][ngrp] fp32 row/group multipliers | mbarriers | abort flag | boundaries
+  // smem layout: [NB][R][K] bf16 row buffers | (RESID) [Rs][K] fp32 residual |
+  // (PROJ) [32][K+8] bf16 U^T | (PROJ) [R][32] bf16 -c |
+  // [2][Rs][nblk] fp32 block sum-of-squares | [2][Rs][ngrp] u32 amax bits |
+  // mbarriers | abort flag | boundaries
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
-  size_t off = (size_t)2 * R * K * 2;
+  size_t off = (size_t)NB * R * K * 2;
   float* xr = nullptr;
-  float* cf = nullptr;
-  uint32_t* up = nullptr;
-  if constexpr (PROJ) {
+  uint16_t* ut = nullptr;
+  uint16_t* negc = nullptr;
+  if constexpr (RESID) {
     xr = reinterpret_cast<float*>(smem + off);
-    off += (size_t)R * K * 4;
-    cf = reinterpret_cast<float*>(smem + off);
-    off += (size_t)R * 32 * 4;
-    up = reinterpret_cast<uint32_t*>(smem + off);
-    off += (size_t)(K / 2) * 32 * 4;
+    off += (size_t)Rs * K * 4;
   }
-  // block partials, double-buffered by group parity so that no barrier is
-  // needed between a group's quantization and the next group's reductions
+  if constexpr (PROJ) {
+    ut = reinterpret_cast<uint16_t*>(smem + off);
+    off += (size_t)32 * ut_pitch(K) * 2;
+    negc = reinterpret_cast<uint16_t*>(smem + off);
+    off += (size_t)R * 32 * 2;
+  }
+  // block partials, double-buffered by sub-group parity so that no barrier is
+  // needed between a sub-group's quantization and the next one's reductions
   float* part_ss2 = reinterpret_cast<float*>(smem + off);
-  off += (size_t)2 * R * nblk * 4;
+  off += (size_t)2 * Rs * nblk * 4;
   const int ngrp = (WEIGHT && FMT == RQ_FMT_INT4) ? K / 128 : 1;
   uint32_t* amax_bits2 = reinterpret_cast<uint32_t*>(smem + off);
-  off += (size_t)2 * R * ngrp * 4;
+  off += (size_t)2 * Rs * ngrp * 4;
   off = (off + 15) & ~(size_t)15;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + off + 16);
@@ -119,11 +146,17 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     fence_mbar_init();
   }
   if constexpr (PROJ) {
-    // stage U (K x 32 BF16) once per CTA as words {U[2i][j], U[2i+1][j]}
-    for (int t = threadIdx.x; t < (K / 2) * 32; t += K1_THREADS) {
-      const int k2 = t >> 5, j = t & 31;
-      up[t] = (uint32_t)__ldg(p.U + (size_t)(2 * k2) * 32 + j) |
-              ((uint32_t)__ldg(p.U + (size_t)(2 * k2 + 1) * 32 + j) << 16);
+    // stage U^T once per CTA: row j of U^T holds U[0..K-1][j]
+    const int KP = ut_pitch(K);
+    for (int t = threadIdx.x; t < K * 4; t += K1_THREADS) {
+      const int k = t >> 2, q = t & 3;
+      const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)k * 32) + q);
+      const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        ut[(size_t)(8 * q + 2 * h) * KP + k] = (uint16_t)(ww[h] & 0xFFFFu);
+        ut[(size_t)(8 * q + 2 * h + 1) * KP + k] = (uint16_t)(ww[h] >> 16);
+      }
     }
   }
   __syncthreads();
@@ -138,280 +171,318 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
 
   if (threadIdx.x == 0 && blockIdx.x < p.ngroups) issue_group(blockIdx.x, 0);
 
-  for (int i = threadIdx.x; i < 2 * R * ngrp; i += K1_THREADS) amax_bits2[i] = 0u;
+  for (int i = threadIdx.x; i < 2 * Rs * ngrp; i += K1_THREADS) amax_bits2[i] = 0u;
   int it = 0;
+  int sg = 0;                              // sub-group counter (partials parity)
   for (int g = blockIdx.x; g < p.ngroups; g += gridDim.x, ++it) {
-    const int buf = it & 1;
+    const int buf = PROJ ? 0 : (it & 1);
     const int r0 = g * R;
     const int nr = min(R, p.rows - r0);
-    float* part_ss = part_ss2 + (size_t)buf * R * nblk;
-    uint32_t* amax_bits = amax_bits2 + (size_t)buf * R * ngrp;
-    mbar_wait(&full[buf], (it >> 1) & 1, p.status, ST_TIMEOUT_LOAD, abort_flag);
+    const bool has_next = g + (int)gridDim.x < p.ngroups;
+    mbar_wait(&full[buf], PROJ ? (it & 1) : ((it >> 1) & 1), p.status, ST_TIMEOUT_LOAD, abort_flag);
     // everyone has finished the previous group past this barrier
     __syncthreads();
     if (*abort_flag) break;
-    // prefetch the next group into the other buffer (last read by the previous
-    // group's gather) and clear the other reductions (last read by the previous
-    // group's quantization)
-    if (threadIdx.x == 0 && g + (int)gridDim.x < p.ngroups) {
-      fence_proxy_async_smem();
-      issue_group(g + gridDim.x, buf ^ 1);
+    if constexpr (!PROJ) {
+      // prefetch the next group into the other buffer (last read by the
+      // previous group's gather)
+      if (threadIdx.x == 0 && has_next) {
+        fence_proxy_async_smem();
+        issue_group(g + gridDim.x, buf ^ 1);
+      }
     }
-    for (int i = threadIdx.x; i < R * ngrp; i += K1_THREADS) amax_bits2[(size_t)(buf ^ 1) * R * ngrp + i] = 0u;
     const uint16_t* xg = xs + (size_t)buf * R * K;
 
-    // ------------------------------------------------------------ projection
+    // ------------------------------------------------------------ coefficients
     if constexpr (PROJ) {
-      // rows -> FP32 (exact), the buffer that becomes the residual in place
-      for (int t = threadIdx.x; t < nr * K / 2; t += K1_THREADS) {
-        const uint32_t w2 = reinterpret_cast<const uint32_t*>(xg)[t];
-        reinterpret_cast<float2*>(xr)[t] = make_float2(__uint_as_float(w2 << 16), __uint_as_float(w2 & 0xFFFF0000u));
-      }
-      __syncthreads();
-      // c[row][j] = bf16(sum_k x[row][k] U[k][j]), each sum sequential in k.
-      // Thread -> (pair of rows, j): two independent chains share every U load.
-      const int npair = (nr + 1) >> 1;
-      if (threadIdx.x < npair * 32) {
-        const int j = lane;
-        const int ra = 2 * (threadIdx.x >> 5);
-        const int rb = min(ra + 1, nr - 1);
-        const float4* xa = reinterpret_cast<const float4*>(xr + (size_t)ra * K);
-        const float4* xb = reinterpret_cast<const float4*>(xr + (size_t)rb * K);
+      // c[row][j] = bf16(sum_k x[row][k] U[k][j]), each sum one sequential FP32
+      // chain in k.  Warp w takes rows w and w + 16, lane j the column j.
+      const uint4* uj = reinterpret_cast<const uint4*>(ut + (size_t)lane * ut_pitch(K));
+      const int ra = warp, rb = warp + 16;
+      if (ra < nr) {
+        const uint4* xa = reinterpret_cast<const uint4*>(xg + (size_t)ra * K);
         float acc_a = 0.f, acc_b = 0.f;
+        if (rb < nr) {
+          const uint4* xb = reinterpret_cast<const uint4*>(xg + (size_t)rb * K);
+#pragma unroll 2
+          for (int k8 = 0; k8 < K / 8; ++k8) {
+            const uint4 u = uj[k8], a = xa[k8], b = xb[k8];
+            acc_a = fma_bf16<0, 0>(a.x, u.x, acc_a); acc_b = fma_bf16<0, 0>(b.x, u.x, acc_b);
+            acc_a = fma_bf16<1, 1>(a.x, u.x, acc_a); acc_b = fma_bf16<1, 1>(b.x, u.x, acc_b);
+            acc_a = fma_bf16<0, 0>(a.y, u.y, acc_a); acc_b = fma_bf16<0, 0>(b.y, u.y, acc_b);
+            acc_a = fma_bf16<1, 1>(a.y, u.y, acc_a); acc_b = fma_bf16<1, 1>(b.y, u.y, acc_b);
+            acc_a = fma_bf16<0, 0>(a.z, u.z, acc_a); acc_b = fma_bf16<0, 0>(b.z, u.z, acc_b);
+            acc_a = fma_bf16<1, 1>(a.z, u.z, acc_a); acc_b = fma_bf16<1, 1>(b.z, u.z, acc_b);
+            acc_a = fma_bf16<0, 0>(a.w, u.w, acc_a); acc_b = fma_bf16<0, 0>(b.w, u.w, acc_b);
+            acc_a = fma_bf16<1, 1>(a.w, u.w, acc_a); acc_b = fma_bf16<1, 1>(b.w, u.w, acc_b);
+          }
+          const uint16_t cb = __bfloat16_as_ushort(__float2bfloat16_rn(acc_b));
+          p.coef[(size_t)(r0 + rb) * 32 + lane] = cb;
+          negc[rb * 32 + lane] = cb ^ 0x8000u;
+        } else {
 #pragma unroll 4
-        for (int k4 = 0; k4 < K / 4; ++k4) {
-          const float4 va = xa[k4], vb = xb[k4];
-          const uint32_t u01 = up[(2 * k4) * 32 + j], u23 = up[(2 * k4 + 1) * 32 + j];
-          const float u0 = __uint_as_float(u01 << 16), u1 = __uint_as_float(u01 & 0xFFFF0000u);
-          const float u2 = __uint_as_float(u23 << 16), u3 = __uint_as_float(u23 & 0xFFFF0000u);
-          // every product of two BF16 values is exact in FP32: fma == add of the product
-          acc_a = __fmaf_rn(va.x, u0, acc_a); acc_b = __fmaf_rn(vb.x, u0, acc_b);
-          acc_a = __fmaf_rn(va.y, u1, acc_a); acc_b = __fmaf_rn(vb.y, u1, acc_b);
-          acc_a = __fmaf_rn(va.z, u2, acc_a); acc_b = __fmaf_rn(vb.z, u2, acc_b);
-          acc_a = __fmaf_rn(va.w, u3, acc_a); acc_b = __fmaf_rn(vb.w, u3, acc_b);
+          for (int k8 = 0; k8 < K / 8; ++k8) {
+            const uint4 u = uj[k8], a = xa[k8];
+            acc_a = fma_bf16<0, 0>(a.x, u.x, acc_a);
+            acc_a = fma_bf16<1, 1>(a.x, u.x, acc_a);
+            acc_a = fma_bf16<0, 0>(a.y, u.y, acc_a);
+            acc_a = fma_bf16<1, 1>(a.y, u.y, acc_a);
+            acc_a = fma_bf16<0, 0>(a.z, u.z, acc_a);
+            acc_a = fma_bf16<1, 1>(a.z, u.z, acc_a);
+            acc_a = fma_bf16<0, 0>(a.w, u.w, acc_a);
+            acc_a = fma_bf16<1, 1>(a.w, u.w, acc_a);
+          }
         }
         const uint16_t ca = __bfloat16_as_ushort(__float2bfloat16_rn(acc_a));
-        const uint16_t cb = __bfloat16_as_ushort(__float2bfloat16_rn(acc_b));
-        p.coef[(size_t)(r0 + ra) * 32 + j] = ca;
-        cf[ra * 32 + j] = bf16_bits_to_f32(ca);
-        if (rb != ra) {
-          p.coef[(size_t)(r0 + rb) * 32 + j] = cb;
-          cf[rb * 32 + j] = bf16_bits_to_f32(cb);
-        }
+        p.coef[(size_t)(r0 + ra) * 32 + lane] = ca;
+        negc[ra * 32 + lane] = ca ^ 0x8000u;
       }
       __syncthreads();
-      if constexpr (!WEIGHT) {
-        // residual x - sum_j c_j U[k, j], subtracted in order j = 0..31.
-        // Thread -> one k: U[k][0..31] loaded once, applied to every row.
-        for (int k = threadIdx.x; k < K; k += K1_THREADS) {
-          float u[32];
-          const uint4* urow = reinterpret_cast<const uint4*>(p.U + (size_t)k * 32);
+    }
+
+    const int nsub = (nr + Rs - 1) / Rs;
+    for (int s = 0; s < nsub; ++s, ++sg) {
+      const int rs0 = s * Rs;              // first row of the sub-group inside the group
+      const int ns = min(Rs, nr - rs0);
+      float* part_ss = part_ss2 + (size_t)(sg & 1) * Rs * nblk;
+      uint32_t* amax_bits = amax_bits2 + (size_t)(sg & 1) * Rs * ngrp;
+      // the previous sub-group's quantization has read its partials and amax
+      if (s > 0) __syncthreads();
+
+      // ---------------------------------------------------------- residual
+      if constexpr (RESID) {
+        // x - sum_j c_j U[k, j], subtracted in order j = 0..31.  Work unit =
+        // (k, quad of 4 rows): U[k][0..31] is loaded once for the quad; the 32
+        // units of a warp share the quad (K % 32 == 0), so -c loads broadcast.
+        const int KP = ut_pitch(K);
+        const int nq = (ns + 3) >> 2;
+        for (int u = threadIdx.x; u < nq * K; u += K1_THREADS) {
+          const int q = u / K, k = u - q * K;
+          uint32_t uk[32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 w4 = __ldg(urow + q);
-            const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+          for (int j = 0; j < 32; ++j) uk[j] = ut[(size_t)j * KP + k];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              u[8 * q + 2 * h] = __uint_as_float(ww[h] << 16);
-              u[8 * q + 2 * h + 1] = __uint_as_float(ww[h] & 0xFFFF0000u);
+          for (int rr = 0; rr < 4; ++rr) {
+            const int row = 4 * q + rr;    // sub-group row
+            if (row < ns) {
+              const int ri = rs0 + row;    // group row
+              float v = bf16_bits_to_f32(xg[(size_t)ri * K + k]);
+              const uint4* c4 = reinterpret_cast<const uint4*>(negc + ri * 32);
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const uint4 cc = c4[h];
+                v = fma_bf16<0, 0>(cc.x, uk[8 * h + 0], v);
+                v = fma_bf16<1, 0>(cc.x, uk[8 * h + 1], v);
+                v = fma_bf16<0, 0>(cc.y, uk[8 * h + 2], v);
+                v = fma_bf16<1, 0>(cc.y, uk[8 * h + 3], v);
+                v = fma_bf16<0, 0>(cc.z, uk[8 * h + 4], v);
+                v = fma_bf16<1, 0>(cc.z, uk[8 * h + 5], v);
+                v = fma_bf16<0, 0>(cc.w, uk[8 * h + 6], v);
+                v = fma_bf16<1, 0>(cc.w, uk[8 * h + 7], v);
+              }
+              xr[(size_t)row * K + k] = v;
             }
-          }
-          for (int ri = 0; ri < nr; ++ri) {
-            float v = xr[(size_t)ri * K + k];
-            const float4* c4 = reinterpret_cast<const float4*>(cf + ri * 32);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 cc = c4[q];
-              v = __fmaf_rn(-cc.x, u[4 * q], v);      // exact product
-              v = __fmaf_rn(-cc.y, u[4 * q + 1], v);
-              v = __fmaf_rn(-cc.z, u[4 * q + 2], v);
-              v = __fmaf_rn(-cc.w, u[4 * q + 3], v);
-            }
-            xr[(size_t)ri * K + k] = v;
           }
         }
         __syncthreads();
-      }
-    }
-
-    // ------------------------------------------------------------ phase A
-    // gather, transform, block partials; y stays in registers until phase B
-    const int nitems = nr * nblk;
-    float y[IPW][32];
-#pragma unroll
-    for (int s = 0; s < IPW; ++s) {
-      const int item = slot0 + s * SLOTS;
-      if (item < nitems) {
-        const int ri = item / nblk, bk = item - ri * nblk;
-        const int i0 = bk * B + lq * 32;
-        float* v = y[s];
-        const int4* rp = reinterpret_cast<const int4*>(p.rot + i0);
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const int4 rv = __ldg(rp + e4);
-          const int rr[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int src = rr[q] & 0x7fffffff;
-            float xv;
-            if constexpr (PROJ) xv = xr[(size_t)ri * K + src];
-            else xv = bf16_bits_to_f32(xg[(size_t)ri * K + src]);
-            v[4 * e4 + q] = __uint_as_float(__float_as_uint(xv) ^ ((uint32_t)rr[q] & 0x80000000u));
-          }
-        }
-        // butterflies inside the lane: stride h pairs (e, e+h) with bit h of e clear
-#pragma unroll
-        for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if ((e & h) == 0) {
-              const float a = v[e], b = v[e + h];
-              v[e] = __fadd_rn(a, b);
-              v[e + h] = __fsub_rn(a, b);
-            }
-          }
-        }
-        // butterflies across the L lanes of the group: stride 32m pairs lane j
-        // (bit m clear) with lane j^m; one exact FFMA per element: lower lane
-        // v + o, upper lane o - v (+-1 * v is exact)
-#pragma unroll
-        for (int m = 1; m < L; m <<= 1) {
-          const float sgn = (lq & m) ? -1.0f : 1.0f;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __fmaf_rn(sgn, v[e], __shfl_xor_sync(gmask, v[e], m));
-        }
-        float amax = 0.f;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          v[e] = __fmul_rn(v[e], p.inv_sqrt_b);
-          amax = fmaxf(amax, fabsf(v[e]));
-        }
-        if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-          // perfect pairwise tree: five in-lane levels, then lanes by xor 1, 2, ..
-          float sq[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) sq[e] = __fmul_rn(v[e], v[e]);
-#pragma unroll
-          for (int w = 1; w < 32; w <<= 1) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2 * w) sq[e] = __fadd_rn(sq[e], sq[e + w]);
-          }
-          float ss = sq[0];
-#pragma unroll
-          for (int m = 1; m < L; m <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(gmask, ss, m));
-          if (lq == 0) part_ss[ri * nblk + bk] = ss;
-        } else if constexpr (WEIGHT && FMT == RQ_FMT_INT4) {
-          // one scale per 128 rotated coordinates = 4 lanes
-#pragma unroll
-          for (int m = 1; m < (L < 4 ? L : 4); m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
-          if ((lq & 3) == 0) atomicMax(&amax_bits[ri * ngrp + i0 / 128], __float_as_uint(amax));
-        } else {
-#pragma unroll
-          for (int m = 1; m < L; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
-          if (lq == 0) atomicMax(&amax_bits[ri], __float_as_uint(amax));
+        // the row buffer is free: stream the next group in behind the rotation
+        if (s == nsub - 1 && threadIdx.x == 0 && has_next) {
+          fence_proxy_async_smem();
+          issue_group(g + gridDim.x, 0);
         }
       }
-    }
-    __syncthreads();
 
-    // ------------------------------------------------------------ phase B
+      // ---------------------------------------------------------- phase A
+      // gather, transform, block partials; y stays in registers until phase B
+      const int nitems = ns * nblk;
+      float y[IPW][32];
 #pragma unroll
-    for (int s = 0; s < IPW; ++s) {
-      const int item = slot0 + s * SLOTS;
-      if (item < nitems) {
-        const int ri = item / nblk, bk = item - ri * nblk;
-        const int row = r0 + ri;
-        const int i0 = bk * B + lq * 32;
-        const float* v = y[s];
-        uint32_t pk[4] = {0u, 0u, 0u, 0u};   // 32 codes, nibble e at bits 4(e%8) of word e/8
-        // row (or group) scale, derived by every lane from the block partials;
-        // the first lane of the row's (group's) first block writes it out
-        float mlt;
-        if constexpr (FMT == RQ_FMT_INT4) {
-          const float amax = __uint_as_float(amax_bits[ri * ngrp + (WEIGHT ? i0 / 128 : 0)]);
-          mlt = amax > 0.f ? __fdiv_rn(7.0f, amax) : 0.f;
-          if (WEIGHT ? (i0 % 128 == 0) : (bk == 0 && lq == 0)) {
-            const float sc = amax > 0.f ? __fdiv_rn(amax, 7.0f) : 0.f;
-            if constexpr (WEIGHT) p.scale[(size_t)(i0 / 128) * p.rows + row] = sc;
-            else p.scale[row] = sc;
+      for (int sl = 0; sl < IPW; ++sl) {
+        const int item = slot0 + sl * SLOTS;
+        if (item < nitems) {
+          const int ri = item / nblk, bk = item - ri * nblk;
+          const int i0 = bk * B + lq * 32;
+          float* v = y[sl];
+          const int4* rp = reinterpret_cast<const int4*>(p.rot + i0);
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const int4 rv = __ldg(rp + e4);
+            const int rr[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int src = rr[q] & 0x7fffffff;
+              float xv;
+              if constexpr (RESID) xv = xr[(size_t)ri * K + src];
+              else xv = bf16_bits_to_f32(xg[(size_t)(rs0 + ri) * K + src]);
+              v[4 * e4 + q] = __uint_as_float(__float_as_uint(xv) ^ ((uint32_t)rr[q] & 0x80000000u));
+            }
           }
-        } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-          float ss = part_ss[ri * nblk];
-          for (int j = 1; j < nblk; ++j) ss = __fadd_rn(ss, part_ss[ri * nblk + j]);
-          const float nrm = __fsqrt_rn(ss);
-          mlt = nrm > 0.f ? __fdiv_rn(p.sqrtK, nrm) : 0.f;
-          if (bk == 0 && lq == 0) p.scale[row] = nrm > 0.f ? __fdiv_rn(nrm, p.sqrtK) : 0.f;
-        } else {
-          const float amax = __uint_as_float(amax_bits[ri]);
-          mlt = amax > 0.f ? __fdiv_rn(2688.0f, amax) : 0.f;
-          if (bk == 0 && lq == 0) p.scale[row] = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 0.f;
-        }
-        if constexpr (FMT == RQ_FMT_INT4) {
-          const float inv = mlt;
+          // butterflies inside the lane: stride h pairs (e, e+h) with bit h of e clear
+#pragma unroll
+          for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if ((e & h) == 0) {
+                const float a = v[e], b = v[e + h];
+                v[e] = __fadd_rn(a, b);
+                v[e + h] = __fsub_rn(a, b);
+              }
+            }
+          }
+          // butterflies across the L lanes of the group: stride 32m pairs lane j
+          // (bit m clear) with lane j^m; one exact FFMA per element: lower lane
+          // v + o, upper lane o - v (+-1 * v is exact)
+#pragma unroll
+          for (int m = 1; m < L; m <<= 1) {
+            const float sgn = (lq & m) ? -1.0f : 1.0f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __fmaf_rn(sgn, v[e], __shfl_xor_sync(gmask, v[e], m));
+          }
+          float amax = 0.f;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            int q = __float2int_rn(__fmul_rn(v[e], inv));
-            q = max(-7, min(7, q));
-            pk[e >> 3] |= ((uint32_t)q & 0xFu) << (4 * (e & 7));
+            v[e] = __fmul_rn(v[e], p.inv_sqrt_b);
+            amax = fmaxf(amax, fabsf(v[e]));
           }
-        } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-          const float inv = mlt;
+          if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+            // perfect pairwise tree: five in-lane levels, then lanes by xor 1, 2, ..
+            float sq[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float u = __fmul_rn(v[e], inv);
-            // number of boundaries <= u (ascending, padded with +inf to 16)
-            uint32_t c = 0;
-            if constexpr (FMT == RQ_FMT_LM16) {
+            for (int e = 0; e < 32; ++e) sq[e] = __fmul_rn(v[e], v[e]);
 #pragma unroll
-              for (int step = 8; step >= 1; step >>= 1)
-                if (u >= bnd_s[c + step - 1]) c += step;
-              pk[e >> 3] |= c << (4 * (e & 7));
-            } else {
-              c = (u >= bnd_s[0]) + (u >= bnd_s[1]) + (u >= bnd_s[2]);
-              pk[e >> 4] |= c << (2 * (e & 15));
+            for (int w = 1; w < 32; w <<= 1) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 2 * w) sq[e] = __fadd_rn(sq[e], sq[e + w]);
             }
+            float ss = sq[0];
+#pragma unroll
+            for (int m = 1; m < L; m <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(gmask, ss, m));
+            if (lq == 0) part_ss[ri * nblk + bk] = ss;
+          } else if constexpr (WEIGHT && FMT == RQ_FMT_INT4) {
+            // one scale per 128 rotated coordinates = 4 lanes
+#pragma unroll
+            for (int m = 1; m < (L < 4 ? L : 4); m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
+            if ((lq & 3) == 0) atomicMax(&amax_bits[ri * ngrp + i0 / 128], __float_as_uint(amax));
+          } else {
+#pragma unroll
+            for (int m = 1; m < L; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
+            if (lq == 0) atomicMax(&amax_bits[ri], __float_as_uint(amax));
           }
-        } else {  // NVFP4: two 16-element groups per lane
-          const float inv_t = mlt;
-          uint16_t sbs = 0;
-#pragma unroll
-          for (int gq = 0; gq < 2; ++gq) {
-            float u[16];
-            float m16 = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              u[e] = __fmul_rn(v[16 * gq + e], inv_t);
-              m16 = fmaxf(m16, fabsf(u[e]));
-            }
-            const float sbf = __fdiv_rn(m16, 6.0f);
-            const uint8_t sb = (uint8_t)(cvt_e4m3x2(0.f, sbf) & 0xFF);
-            const float rcp = sb ? __fdiv_rn(1.0f, e4m3_to_f32(sb)) : 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const uint32_t byte = sb ? (uint32_t)cvt_e2m1x2(__fmul_rn(u[e + 1], rcp), __fmul_rn(u[e], rcp)) : 0u;
-              const int ee = 16 * gq + e;
-              pk[ee >> 3] |= byte << (4 * (ee & 7));
-            }
-            sbs |= (uint16_t)sb << (8 * gq);
-          }
-          // block scales kb, kb+1 (kb even) are adjacent bytes of the tile layout
-          *reinterpret_cast<uint16_t*>(p.bscale + sf_offset(row, i0 / 16, K)) = sbs;
         }
-        if constexpr (FMT == RQ_FMT_LM4) {
-          *reinterpret_cast<uint2*>(p.codes + (size_t)row * (K / 4) + i0 / 4) = make_uint2(pk[0], pk[1]);
-        } else {
-          *reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 2) + i0 / 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      __syncthreads();
+      // the previous sub-group's amax words are free again (its quantization
+      // finished before the barrier above)
+      for (int i = threadIdx.x; i < Rs * ngrp; i += K1_THREADS)
+        amax_bits2[(size_t)((sg & 1) ^ 1) * Rs * ngrp + i] = 0u;
+      if constexpr (PROJ && !RESID) {
+        // weight rows were gathered straight from the row buffer: free now
+        if (s == nsub - 1 && threadIdx.x == 0 && has_next) {
+          fence_proxy_async_smem();
+          issue_group(g + gridDim.x, 0);
+        }
+      }
+
+      // ---------------------------------------------------------- phase B
+#pragma unroll
+      for (int sl = 0; sl < IPW; ++sl) {
+        const int item = slot0 + sl * SLOTS;
+        if (item < nitems) {
+          const int ri = item / nblk, bk = item - ri * nblk;
+          const int row = r0 + rs0 + ri;
+          const int i0 = bk * B + lq * 32;
+          const float* v = y[sl];
+          uint32_t pk[4] = {0u, 0u, 0u, 0u};   // 32 codes, nibble e at bits 4(e%8) of word e/8
+          // row (or group) scale, derived by every lane from the block partials;
+          // the first lane of the row's (group's) first block writes it out
+          float mlt;
+          if constexpr (FMT == RQ_FMT_INT4) {
+            const float amax = __uint_as_float(amax_bits[ri * ngrp + (WEIGHT ? i0 / 128 : 0)]);
+            mlt = amax > 0.f ? __fdiv_rn(7.0f, amax) : 0.f;
+            if (WEIGHT ? (i0 % 128 == 0) : (bk == 0 && lq == 0)) {
+              const float sc = amax > 0.f ? __fdiv_rn(amax, 7.0f) : 0.f;
+              if constexpr (WEIGHT) p.scale[(size_t)(i0 / 128) * p.rows + row] = sc;
+              else p.scale[row] = sc;
+            }
+          } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+            float ss = part_ss[ri * nblk];
+            for (int j = 1; j < nblk; ++j) ss = __fadd_rn(ss, part_ss[ri * nblk + j]);
+            const float nrm = __fsqrt_rn(ss);
+            mlt = nrm > 0.f ? __fdiv_rn(p.sqrtK, nrm) : 0.f;
+            if (bk == 0 && lq == 0) p.scale[row] = nrm > 0.f ? __fdiv_rn(nrm, p.sqrtK) : 0.f;
+          } else {
+            const float amax = __uint_as_float(amax_bits[ri]);
+            mlt = amax > 0.f ? __fdiv_rn(2688.0f, amax) : 0.f;
+            if (bk == 0 && lq == 0) p.scale[row] = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 0.f;
+          }
+          if constexpr (FMT == RQ_FMT_INT4) {
+            const float inv = mlt;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              int q = __float2int_rn(__fmul_rn(v[e], inv));
+              q = max(-7, min(7, q));
+              pk[e >> 3] |= ((uint32_t)q & 0xFu) << (4 * (e & 7));
+            }
+          } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+            const float inv = mlt;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float u = __fmul_rn(v[e], inv);
+              // number of boundaries <= u (ascending, padded with +inf to 16)
+              uint32_t c = 0;
+              if constexpr (FMT == RQ_FMT_LM16) {
+#pragma unroll
+                for (int step = 8; step >= 1; step >>= 1)
+                  if (u >= bnd_s[c + step - 1]) c += step;
+                pk[e >> 3] |= c << (4 * (e & 7));
+              } else {
+                c = (u >= bnd_s[0]) + (u >= bnd_s[1]) + (u >= bnd_s[2]);
+                pk[e >> 4] |= c << (2 * (e & 15));
+              }
+            }
+          } else {  // NVFP4: two 16-element groups per lane
+            const float inv_t = mlt;
+            uint16_t sbs = 0;
+#pragma unroll
+            for (int gq = 0; gq < 2; ++gq) {
+              float u[16];
+              float m16 = 0.f;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                u[e] = __fmul_rn(v[16 * gq + e], inv_t);
+                m16 = fmaxf(m16, fabsf(u[e]));
+              }
+              const float sbf = __fdiv_rn(m16, 6.0f);
+              const uint8_t sb = (uint8_t)(cvt_e4m3x2(0.f, sbf) & 0xFF);
+              const float rcp = sb ? __fdiv_rn(1.0f, e4m3_to_f32(sb)) : 0.f;
+#pragma unroll
+              for (int e = 0; e < 16; e += 2) {
+                const uint32_t byte = sb ? (uint32_t)cvt_e2m1x2(__fmul_rn(u[e + 1], rcp), __fmul_rn(u[e], rcp)) : 0u;
+                const int ee = 16 * gq + e;
+                pk[ee >> 3] |= byte << (4 * (ee & 7));
+              }
+              sbs |= (uint16_t)sb << (8 * gq);
+            }
+            // block scales kb, kb+1 (kb even) are adjacent bytes of the tile layout
+            *reinterpret_cast<uint16_t*>(p.bscale + sf_offset(row, i0 / 16, K)) = sbs;
+          }
+          if constexpr (FMT == RQ_FMT_LM4) {
+            *reinterpret_cast<uint2*>(p.codes + (size_t)row * (K / 4) + i0 / 4) = make_uint2(pk[0], pk[1]);
+          } else {
+            *reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 2) + i0 / 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
         }
       }
     }
   }
 }
 
-size_t k1_smem_bytes(int R, int K, int nblk, bool proj, int ngrp) {
-  size_t off = (size_t)2 * R * K * 2;
-  if (proj) off += (size_t)R * K * 4 + (size_t)R * 32 * 4 + (size_t)(K / 2) * 32 * 4;
-  off += (size_t)2 * R * nblk * 4;
-  off += (size_t)2 * R * ngrp * 4;
+size_t k1_smem_bytes(int R, int Rs, int K, int nblk, bool proj, bool resid, int ngrp) {
+  size_t off = (size_t)(proj ? 1 : 2) * R * K * 2;
+  if (resid) off += (size_t)Rs * K * 4;
+  if (proj) off += (size_t)32 * ut_pitch(K) * 2 + (size_t)R * 32 * 2;
+  off += (size_t)2 * Rs * nblk * 4;
+  off += (size_t)2 * Rs * ngrp * 4;
   off = (off + 15) & ~(size_t)15;
   return off + 32 + 64;
 }
@@ -436,26 +507,52 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
   p.nbnd = a.nbnd;
   for (int i = 0; i < 15; ++i) p.bnd[i] = i < a.nbnd ? a.bnd[i] : 0.f;
   const int nblk = a.K / (L * 32);
-  // rows per group: as many as fill IPW passes of the block slots
-  int R = (SLOTS * IPW) / nblk;
-  if (R < 1) return cudaErrorInvalidValue;
-  if (R > 24) R = 24;
-  if (PROJ && R > 12) R = 12;
   const int ngrp = (WEIGHT && FMT == RQ_FMT_INT4) ? a.K / 128 : 1;
-  size_t smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp);
-  // two CTAs per SM for the single-pass variant
-  const size_t cap = IPW == 1 ? 110 * 1024 : 200 * 1024;
-  while (smem > cap && R > 1) {
-    --R;
-    smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp);
+  const int sms = a.num_sms > 0 ? a.num_sms : 148;
+  int R = 0, Rs = 0;
+  size_t smem = 0;
+  if constexpr (PROJ) {
+    // one load of R rows per CTA and wave (at most 32: two coefficient chains
+    // per thread), rotated in sub-groups of at most 16 rows that fit the slots
+    const size_t cap = 232448;
+    int R0 = (a.rows + sms - 1) / sms;
+    R0 = R0 < 1 ? 1 : (R0 > 32 ? 32 : R0);
+    for (int r = R0; r >= 1 && !R; --r) {
+      for (int nsub = (r + 15) / 16; nsub <= r; ++nsub) {
+        const int rs = (r + nsub - 1) / nsub;
+        if (rs * nblk > SLOTS * IPW) continue;
+        const size_t b = k1_smem_bytes(r, rs, a.K, nblk, true, !WEIGHT, ngrp);
+        if (b <= cap) {
+          R = r;
+          Rs = rs;
+          smem = b;
+          break;
+        }
+      }
+    }
+    if (!R) return cudaErrorInvalidValue;
+  } else {
+    // rows per group: as many as fill IPW passes of the block slots
+    R = (SLOTS * IPW) / nblk;
+    if (R < 1) return cudaErrorInvalidValue;
+    if (R > 24) R = 24;
+    smem = k1_smem_bytes(R, R, a.K, nblk, false, false, ngrp);
+    // two CTAs per SM for the single-pass variant
+    const size_t cap = IPW == 1 ? 110 * 1024 : 200 * 1024;
+    while (smem > cap && R > 1) {
+      --R;
+      smem = k1_smem_bytes(R, R, a.K, nblk, false, false, ngrp);
+    }
+    if (smem > cap) return cudaErrorInvalidValue;
+    Rs = R;
   }
-  if (smem > cap) return cudaErrorInvalidValue;
   p.R = R;
+  p.Rs = Rs;
   p.ngroups = (a.rows + R - 1) / R;
   auto kern = k1_rotate_quantize<L, FMT, PROJ, WEIGHT, IPW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int grid = (a.num_sms > 0 ? a.num_sms : 148) * (IPW == 1 ? 2 : 1);
+  int grid = sms * (IPW == 1 ? 2 : 1);
   if (grid > p.ngroups) grid = p.ngroups;
   kern<<<grid, K1_THREADS, smem, st>>>(p);
   return cudaGetLastError();
