@@ -9,9 +9,9 @@
 //
 // Data flow per CTA (persistent over groups of R rows):
 //   HBM --cp.async.bulk--> smem row buffer (mbarrier)
-//   [projection: c = bf16(x U), each of the R x 32 sums a sequential FP32 chain
-//    over k (one chain per thread, every warp busy); then, in sub-groups of Rs
-//    rows, x_res = x - c U^T (sequential over j) into an FP32 buffer]
+//   [projection: c = bf16(x U) from the BF16 rows, each of the R x 32 sums a
+//    sequential FP32 chain over k; the rows are widened to FP32 in place and
+//    x_res = x - c U^T (sequential over j) overwrites them]
 //   a group of L = b/32 lanes owns one b-wide Hadamard block of one row: lane j
 //   of the group holds the 32 consecutive rotated coordinates 32j .. 32j+31,
 //   gathered from smem through the signed-permutation table; butterfly stages
@@ -23,9 +23,7 @@
 // FP32 contract (bit-exact against the CPU oracle): every add/multiply/divide is
 // an explicit round-to-nearest-even intrinsic (no contraction); the only fused
 // multiply-adds are the projection's, whose products of two BF16 values are
-// exact in FP32 so the fused and unfused results agree.  They are issued as
-// fma.rn.f32.bf16 (BF16 operands, FP32 addend and result), which is the same
-// single rounding of the exact product plus the addend.
+// exact in FP32 so the fused and unfused results agree.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -52,8 +50,7 @@ struct __align__(16) K1Params {
   uint8_t* bscale;         // NVFP4 block scales, 128x4 swizzled tiles
   int32_t* status;
   int32_t rows, K, r;
-  int32_t R;               // rows per group (one load)
-  int32_t Rs;              // rows per sub-group (rotation / quantization pass)
+  int32_t R;               // rows per group
   int32_t ngroups;
   float inv_sqrt_b;        // fp32(1/sqrt(block))
   float sqrtK;             // fp32(sqrt(K))
@@ -87,16 +84,16 @@ __device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float acc) {
 // (the 16-byte pad spreads the 32 rows over all banks).
 __host__ __device__ constexpr int ut_pitch(int K) { return K + 8; }
 
+
 template <int L, int FMT, bool PROJ, bool WEIGHT, int IPW>
 __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quantize(const __grid_constant__ K1Params p) {
   constexpr int B = L * 32;                // Hadamard block
   constexpr int GPW = 32 / L;              // lane groups (block slots) per warp
   constexpr int SLOTS = K1_WARPS * GPW;    // block slots per CTA pass
   constexpr bool RESID = PROJ && !WEIGHT;  // activations: rotate the residual
-  constexpr int NB = PROJ ? 1 : 2;         // row buffers (prefetch without projection)
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = p.K;
-  const int R = p.R, Rs = p.Rs;
+  const int R = p.R;
   const int nblk = K / B;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -105,32 +102,39 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
   // shuffles stay inside the lane group (groups of one warp may take different branches)
   const unsigned gmask = L == 32 ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
 
-  // smem layout: [NB][R][K] bf16 row buffers | (RESID) [Rs][K] fp32 residual |
-  // (PROJ) [32][K+8] bf16 U^T | (PROJ) [R][32] bf16 -c |
-  // [2][Rs][nblk] fp32 block sum-of-squares | [2][Rs][ngrp] u32 amax bits |
-  // mbarriers | abort flag | boundaries
+  // smem layout
+  //   without projection: [2][R][K] bf16 row buffers (the next group streams in
+  //   while this one is transformed)
+  //   with projection: [R][K] fp32 rows (the bf16 rows land in its upper half
+  //   and are widened in place) | [32][K+8] bf16 U^T | [R][32] fp32 -c |
+  //   [K] int32 signed permutation
+  //   then [2][R][nblk] fp32 block sum-of-squares | [2][R][ngrp] u32 amax bits |
+  //   mbarriers | abort flag | boundaries
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
-  size_t off = (size_t)NB * R * K * 2;
-  float* xr = nullptr;
+  float* xf = reinterpret_cast<float*>(smem);
+  uint16_t* land = reinterpret_cast<uint16_t*>(smem + (PROJ ? (size_t)R * K * 2 : 0));
+  size_t off;
   uint16_t* ut = nullptr;
-  uint16_t* negc = nullptr;
-  if constexpr (RESID) {
-    xr = reinterpret_cast<float*>(smem + off);
-    off += (size_t)Rs * K * 4;
-  }
+  float* negc = nullptr;
+  int32_t* rot_s = nullptr;
   if constexpr (PROJ) {
+    off = (size_t)R * K * 4;
     ut = reinterpret_cast<uint16_t*>(smem + off);
     off += (size_t)32 * ut_pitch(K) * 2;
-    negc = reinterpret_cast<uint16_t*>(smem + off);
-    off += (size_t)R * 32 * 2;
+    negc = reinterpret_cast<float*>(smem + off);
+    off += (size_t)R * 32 * 4;
+    rot_s = reinterpret_cast<int32_t*>(smem + off);
+    off += (size_t)K * 4;
+  } else {
+    off = (size_t)2 * R * K * 2;
   }
-  // block partials, double-buffered by sub-group parity so that no barrier is
-  // needed between a sub-group's quantization and the next one's reductions
+  // block partials, double-buffered by group parity so that no barrier is
+  // needed between a group's quantization and the next group's reductions
   float* part_ss2 = reinterpret_cast<float*>(smem + off);
-  off += (size_t)2 * Rs * nblk * 4;
+  off += (size_t)2 * R * nblk * 4;
   const int ngrp = (WEIGHT && FMT == RQ_FMT_INT4) ? K / 128 : 1;
   uint32_t* amax_bits2 = reinterpret_cast<uint32_t*>(smem + off);
-  off += (size_t)2 * Rs * ngrp * 4;
+  off += (size_t)2 * R * ngrp * 4;
   off = (off + 15) & ~(size_t)15;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + off + 16);
@@ -145,8 +149,21 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     *abort_flag = 0;
     fence_mbar_init();
   }
+  __syncthreads();
+
+  auto issue_group = [&](int g, int buf) {
+    const int r0 = g * R;
+    const int nr = min(R, p.rows - r0);
+    uint16_t* dst = PROJ ? land : xs + (size_t)buf * R * K;
+    mbar_expect_tx(&full[buf], (uint32_t)nr * row_bytes);
+    for (int i = 0; i < nr; ++i) bulk_g2s(dst + (size_t)i * K, p.x + (size_t)(r0 + i) * K, row_bytes, &full[buf]);
+  };
+
+  if (threadIdx.x == 0 && blockIdx.x < p.ngroups) issue_group(blockIdx.x, 0);
+
   if constexpr (PROJ) {
-    // stage U^T once per CTA: row j of U^T holds U[0..K-1][j]
+    // stage U^T (row j holds U[0..K-1][j]) and the signed permutation once per
+    // CTA, while the first rows stream in
     const int KP = ut_pitch(K);
     for (int t = threadIdx.x; t < K * 4; t += K1_THREADS) {
       const int k = t >> 2, q = t & 3;
@@ -158,27 +175,19 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
         ut[(size_t)(8 * q + 2 * h + 1) * KP + k] = (uint16_t)(ww[h] >> 16);
       }
     }
+    for (int t = threadIdx.x; t < K / 4; t += K1_THREADS)
+      reinterpret_cast<int4*>(rot_s)[t] = __ldg(reinterpret_cast<const int4*>(p.rot) + t);
   }
-  __syncthreads();
 
-  auto issue_group = [&](int g, int buf) {
-    const int r0 = g * R;
-    const int nr = min(R, p.rows - r0);
-    mbar_expect_tx(&full[buf], (uint32_t)nr * row_bytes);
-    for (int i = 0; i < nr; ++i)
-      bulk_g2s(xs + ((size_t)buf * R + i) * K, p.x + (size_t)(r0 + i) * K, row_bytes, &full[buf]);
-  };
-
-  if (threadIdx.x == 0 && blockIdx.x < p.ngroups) issue_group(blockIdx.x, 0);
-
-  for (int i = threadIdx.x; i < 2 * Rs * ngrp; i += K1_THREADS) amax_bits2[i] = 0u;
+  for (int i = threadIdx.x; i < 2 * R * ngrp; i += K1_THREADS) amax_bits2[i] = 0u;
   int it = 0;
-  int sg = 0;                              // sub-group counter (partials parity)
   for (int g = blockIdx.x; g < p.ngroups; g += gridDim.x, ++it) {
     const int buf = PROJ ? 0 : (it & 1);
     const int r0 = g * R;
     const int nr = min(R, p.rows - r0);
     const bool has_next = g + (int)gridDim.x < p.ngroups;
+    float* part_ss = part_ss2 + (size_t)(it & 1) * R * nblk;
+    uint32_t* amax_bits = amax_bits2 + (size_t)(it & 1) * R * ngrp;
     mbar_wait(&full[buf], PROJ ? (it & 1) : ((it >> 1) & 1), p.status, ST_TIMEOUT_LOAD, abort_flag);
     // everyone has finished the previous group past this barrier
     __syncthreads();
@@ -193,296 +202,363 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     }
     const uint16_t* xg = xs + (size_t)buf * R * K;
 
-    // ------------------------------------------------------------ coefficients
     if constexpr (PROJ) {
+      // ---------------------------------------------------------- coefficients
       // c[row][j] = bf16(sum_k x[row][k] U[k][j]), each sum one sequential FP32
-      // chain in k.  Warp w takes rows w and w + 16, lane j the column j.
-      const uint4* uj = reinterpret_cast<const uint4*>(ut + (size_t)lane * ut_pitch(K));
-      const int ra = warp, rb = warp + 16;
-      if (ra < nr) {
-        const uint4* xa = reinterpret_cast<const uint4*>(xg + (size_t)ra * K);
-        float acc_a = 0.f, acc_b = 0.f;
-        if (rb < nr) {
-          const uint4* xb = reinterpret_cast<const uint4*>(xg + (size_t)rb * K);
+      // chain in k, read straight from the BF16 rows as they landed.  Warp w
+      // takes rows w and w + 16 (two interleaved chains), lane j the column j.
+      // fma.rn.f32.bf16 rounds the exact product plus the addend once, like
+      // an FMA on the widened operands.
+      if (warp < nr) {
+        const bool two = warp + 16 < nr;
+        const uint4* uj = reinterpret_cast<const uint4*>(ut + (size_t)lane * ut_pitch(K));
+        const uint4* xa = reinterpret_cast<const uint4*>(land + (size_t)warp * K);
+        const uint4* xb = reinterpret_cast<const uint4*>(land + (size_t)(two ? warp + 16 : warp) * K);
+        float ca = 0.f, cb = 0.f;
 #pragma unroll 2
-          for (int k8 = 0; k8 < K / 8; ++k8) {
-            const uint4 u = uj[k8], a = xa[k8], b = xb[k8];
-            acc_a = fma_bf16<0, 0>(a.x, u.x, acc_a); acc_b = fma_bf16<0, 0>(b.x, u.x, acc_b);
-            acc_a = fma_bf16<1, 1>(a.x, u.x, acc_a); acc_b = fma_bf16<1, 1>(b.x, u.x, acc_b);
-            acc_a = fma_bf16<0, 0>(a.y, u.y, acc_a); acc_b = fma_bf16<0, 0>(b.y, u.y, acc_b);
-            acc_a = fma_bf16<1, 1>(a.y, u.y, acc_a); acc_b = fma_bf16<1, 1>(b.y, u.y, acc_b);
-            acc_a = fma_bf16<0, 0>(a.z, u.z, acc_a); acc_b = fma_bf16<0, 0>(b.z, u.z, acc_b);
-            acc_a = fma_bf16<1, 1>(a.z, u.z, acc_a); acc_b = fma_bf16<1, 1>(b.z, u.z, acc_b);
-            acc_a = fma_bf16<0, 0>(a.w, u.w, acc_a); acc_b = fma_bf16<0, 0>(b.w, u.w, acc_b);
-            acc_a = fma_bf16<1, 1>(a.w, u.w, acc_a); acc_b = fma_bf16<1, 1>(b.w, u.w, acc_b);
-          }
-          const uint16_t cb = __bfloat16_as_ushort(__float2bfloat16_rn(acc_b));
-          p.coef[(size_t)(r0 + rb) * 32 + lane] = cb;
-          negc[rb * 32 + lane] = cb ^ 0x8000u;
-        } else {
-#pragma unroll 4
-          for (int k8 = 0; k8 < K / 8; ++k8) {
-            const uint4 u = uj[k8], a = xa[k8];
-            acc_a = fma_bf16<0, 0>(a.x, u.x, acc_a);
-            acc_a = fma_bf16<1, 1>(a.x, u.x, acc_a);
-            acc_a = fma_bf16<0, 0>(a.y, u.y, acc_a);
-            acc_a = fma_bf16<1, 1>(a.y, u.y, acc_a);
-            acc_a = fma_bf16<0, 0>(a.z, u.z, acc_a);
-            acc_a = fma_bf16<1, 1>(a.z, u.z, acc_a);
-            acc_a = fma_bf16<0, 0>(a.w, u.w, acc_a);
-            acc_a = fma_bf16<1, 1>(a.w, u.w, acc_a);
-          }
+        for (int k8 = 0; k8 < K / 8; ++k8) {
+          const uint4 u = uj[k8], a = xa[k8], b = xb[k8];
+          ca = fma_bf16<0, 0>(a.x, u.x, ca); cb = fma_bf16<0, 0>(b.x, u.x, cb);
+          ca = fma_bf16<1, 1>(a.x, u.x, ca); cb = fma_bf16<1, 1>(b.x, u.x, cb);
+          ca = fma_bf16<0, 0>(a.y, u.y, ca); cb = fma_bf16<0, 0>(b.y, u.y, cb);
+          ca = fma_bf16<1, 1>(a.y, u.y, ca); cb = fma_bf16<1, 1>(b.y, u.y, cb);
+          ca = fma_bf16<0, 0>(a.z, u.z, ca); cb = fma_bf16<0, 0>(b.z, u.z, cb);
+          ca = fma_bf16<1, 1>(a.z, u.z, ca); cb = fma_bf16<1, 1>(b.z, u.z, cb);
+          ca = fma_bf16<0, 0>(a.w, u.w, ca); cb = fma_bf16<0, 0>(b.w, u.w, cb);
+          ca = fma_bf16<1, 1>(a.w, u.w, ca); cb = fma_bf16<1, 1>(b.w, u.w, cb);
         }
-        const uint16_t ca = __bfloat16_as_ushort(__float2bfloat16_rn(acc_a));
-        p.coef[(size_t)(r0 + ra) * 32 + lane] = ca;
-        negc[ra * 32 + lane] = ca ^ 0x8000u;
+        const uint16_t ha = __bfloat16_as_ushort(__float2bfloat16_rn(ca));
+        p.coef[(size_t)(r0 + warp) * 32 + lane] = ha;
+        negc[warp * 32 + lane] = -bf16_bits_to_f32(ha);
+        if (two) {
+          const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(cb));
+          p.coef[(size_t)(r0 + warp + 16) * 32 + lane] = hb;
+          negc[(warp + 16) * 32 + lane] = -bf16_bits_to_f32(hb);
+        }
       }
       __syncthreads();
-    }
 
-    const int nsub = (nr + Rs - 1) / Rs;
-    for (int s = 0; s < nsub; ++s, ++sg) {
-      const int rs0 = s * Rs;              // first row of the sub-group inside the group
-      const int ns = min(Rs, nr - rs0);
-      float* part_ss = part_ss2 + (size_t)(sg & 1) * Rs * nblk;
-      uint32_t* amax_bits = amax_bits2 + (size_t)(sg & 1) * Rs * ngrp;
-      // the previous sub-group's quantization has read its partials and amax
-      if (s > 0) __syncthreads();
+      // ---------------------------------------------------------- widen
+      // BF16 -> FP32 in place (exact).  A stage converts the rows [u, v) whose
+      // FP32 targets end before landing row u; the last row overlaps its own
+      // landing row and goes through registers.
+      {
+        const uint32_t* land32 = reinterpret_cast<const uint32_t*>(land);
+        int u = 0;
+        while (u < nr) {
+          const int v = min(nr, (R + u) >> 1);
+          if (v > u) {
+            for (int t = threadIdx.x; t < (v - u) * K / 2; t += K1_THREADS) {
+              const uint32_t w2 = land32[(size_t)u * K / 2 + t];
+              reinterpret_cast<float2*>(xf)[(size_t)u * K / 2 + t] =
+                  make_float2(__uint_as_float(w2 << 16), __uint_as_float(w2 & 0xFFFF0000u));
+            }
+            u = v;
+          } else {
+            uint32_t w[4];   // K <= 3072: at most three words per thread
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int t = threadIdx.x + i * K1_THREADS;
+              if (t < K / 2) w[i] = land32[(size_t)u * K / 2 + t];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int t = threadIdx.x + i * K1_THREADS;
+              if (t < K / 2)
+                reinterpret_cast<float2*>(xf)[(size_t)u * K / 2 + t] =
+                    make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+            }
+            u = u + 1;
+          }
+          __syncthreads();
+        }
+      }
 
       // ---------------------------------------------------------- residual
       if constexpr (RESID) {
-        // x - sum_j c_j U[k, j], subtracted in order j = 0..31.  Work unit =
-        // (k, quad of 4 rows): U[k][0..31] is loaded once for the quad; the 32
-        // units of a warp share the quad (K % 32 == 0), so -c loads broadcast.
+        // x - sum_j c_j U[k, j] in place, subtracted in order j = 0..31.  Work
+        // unit = (k pair, one of eight row sets): U[k..k+1][0..31] is widened
+        // once per unit and each broadcast -c load serves both k; the units of
+        // a warp share the row set (K % 64 == 0).  4K units: the same count for
+        // every thread.
         const int KP = ut_pitch(K);
-        const int nq = (ns + 3) >> 2;
-        for (int u = threadIdx.x; u < nq * K; u += K1_THREADS) {
-          const int q = u / K, k = u - q * K;
-          uint32_t uk[32];
+        const int RU = (nr + 7) >> 3;
+        const int KH = K / 2;
+        for (int uu = threadIdx.x; uu < 8 * KH; uu += K1_THREADS) {
+          const int set = uu / KH, k = 2 * (uu - set * KH);
+          const int ra = set * RU, rb = min(nr, ra + RU);
+          if (ra >= rb) continue;
+          // j outermost in blocks of four, the unit's rows (at most four) inner:
+          // every (row, k) chain still runs j = 0..31 in order.  The next
+          // block's U^T words and -c vectors are loaded one block ahead.
+          const int n = rb - ra;
+          const float4* c4[4];
+          float va[4], vb[4];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) uk[j] = ut[(size_t)j * KP + k];
+          for (int r = 0; r < 4; ++r) {
+            const int rr = ra + (r < n ? r : 0);
+            c4[r] = reinterpret_cast<const float4*>(negc + rr * 32);
+            const float2 x2 = *reinterpret_cast<const float2*>(xf + (size_t)rr * K + k);
+            va[r] = x2.x;
+            vb[r] = x2.y;
+          }
+          const uint16_t* uk = ut + k;
+          uint32_t wn[4];
+          float4 cn[4];
 #pragma unroll
-          for (int rr = 0; rr < 4; ++rr) {
-            const int row = 4 * q + rr;    // sub-group row
-            if (row < ns) {
-              const int ri = rs0 + row;    // group row
-              float v = bf16_bits_to_f32(xg[(size_t)ri * K + k]);
-              const uint4* c4 = reinterpret_cast<const uint4*>(negc + ri * 32);
+          for (int i = 0; i < 4; ++i) wn[i] = *reinterpret_cast<const uint32_t*>(uk + (size_t)i * KP);
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const uint4 cc = c4[h];
-                v = fma_bf16<0, 0>(cc.x, uk[8 * h + 0], v);
-                v = fma_bf16<1, 0>(cc.x, uk[8 * h + 1], v);
-                v = fma_bf16<0, 0>(cc.y, uk[8 * h + 2], v);
-                v = fma_bf16<1, 0>(cc.y, uk[8 * h + 3], v);
-                v = fma_bf16<0, 0>(cc.z, uk[8 * h + 4], v);
-                v = fma_bf16<1, 0>(cc.z, uk[8 * h + 5], v);
-                v = fma_bf16<0, 0>(cc.w, uk[8 * h + 6], v);
-                v = fma_bf16<1, 0>(cc.w, uk[8 * h + 7], v);
-              }
-              xr[(size_t)row * K + k] = v;
+          for (int r = 0; r < 4; ++r) cn[r] = c4[r][0];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float ua[4], ub[4];
+            float4 cc[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              ua[i] = __uint_as_float(wn[i] << 16);
+              ub[i] = __uint_as_float(wn[i] & 0xFFFF0000u);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) cc[r] = cn[r];
+            if (q < 7) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) wn[i] = *reinterpret_cast<const uint32_t*>(uk + (size_t)(4 * q + 4 + i) * KP);
+#pragma unroll
+              for (int r = 0; r < 4; ++r) cn[r] = c4[r][q + 1];
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              va[r] = __fmaf_rn(cc[r].x, ua[0], va[r]);     // exact products
+              vb[r] = __fmaf_rn(cc[r].x, ub[0], vb[r]);
+              va[r] = __fmaf_rn(cc[r].y, ua[1], va[r]);
+              vb[r] = __fmaf_rn(cc[r].y, ub[1], vb[r]);
+              va[r] = __fmaf_rn(cc[r].z, ua[2], va[r]);
+              vb[r] = __fmaf_rn(cc[r].z, ub[2], vb[r]);
+              va[r] = __fmaf_rn(cc[r].w, ua[3], va[r]);
+              vb[r] = __fmaf_rn(cc[r].w, ub[3], vb[r]);
             }
           }
+          // rows past the set's end computed a copy of its first row: not stored
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            if (r < n) *reinterpret_cast<float2*>(xf + (size_t)(ra + r) * K + k) = make_float2(va[r], vb[r]);
         }
         __syncthreads();
-        // the row buffer is free: stream the next group in behind the rotation
-        if (s == nsub - 1 && threadIdx.x == 0 && has_next) {
-          fence_proxy_async_smem();
-          issue_group(g + gridDim.x, 0);
-        }
       }
+    }
 
-      // ---------------------------------------------------------- phase A
-      // gather, transform, block partials; y stays in registers until phase B
-      const int nitems = ns * nblk;
-      float y[IPW][32];
+    // ------------------------------------------------------------ phase A
+    // gather, transform, block partials; y stays in registers until phase B
+    const int nitems = nr * nblk;
+    float y[IPW][32];
+    float red[IPW];   // the lane's block partial per item
+    // with two items the partials go out after both items' loads were issued
+    // (a shared store before them would order the second item's gathers behind it)
+    auto publish = [&](int ri, int bk, float val) {
+      if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+        if (lq == 0) part_ss[ri * nblk + bk] = val;
+      } else if constexpr (WEIGHT && FMT == RQ_FMT_INT4) {
+        if ((lq & 3) == 0) atomicMax(&amax_bits[ri * ngrp + (bk * B + lq * 32) / 128], __float_as_uint(val));
+      } else {
+        if (lq == 0) atomicMax(&amax_bits[ri], __float_as_uint(val));
+      }
+    };
 #pragma unroll
-      for (int sl = 0; sl < IPW; ++sl) {
-        const int item = slot0 + sl * SLOTS;
-        if (item < nitems) {
-          const int ri = item / nblk, bk = item - ri * nblk;
-          const int i0 = bk * B + lq * 32;
-          float* v = y[sl];
-          const int4* rp = reinterpret_cast<const int4*>(p.rot + i0);
+    for (int s = 0; s < IPW; ++s) {
+      const int item = slot0 + s * SLOTS;
+      if (item < nitems) {
+        const int ri = item / nblk, bk = item - ri * nblk;
+        const int i0 = bk * B + lq * 32;
+        float* v = y[s];
+        const int4* rp = reinterpret_cast<const int4*>((PROJ ? rot_s : p.rot) + i0);
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const int4 rv = __ldg(rp + e4);
-            const int rr[4] = {rv.x, rv.y, rv.z, rv.w};
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const int4 rv = PROJ ? rp[e4] : __ldg(rp + e4);
+          const int rr[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int src = rr[q] & 0x7fffffff;
-              float xv;
-              if constexpr (RESID) xv = xr[(size_t)ri * K + src];
-              else xv = bf16_bits_to_f32(xg[(size_t)(rs0 + ri) * K + src]);
-              v[4 * e4 + q] = __uint_as_float(__float_as_uint(xv) ^ ((uint32_t)rr[q] & 0x80000000u));
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int src = rr[q] & 0x7fffffff;
+            float xv;
+            if constexpr (PROJ) xv = xf[(size_t)ri * K + src];
+            else xv = bf16_bits_to_f32(xg[(size_t)ri * K + src]);
+            v[4 * e4 + q] = __uint_as_float(__float_as_uint(xv) ^ ((uint32_t)rr[q] & 0x80000000u));
           }
-          // butterflies inside the lane: stride h pairs (e, e+h) with bit h of e clear
+        }
+        // butterflies inside the lane: stride h pairs (e, e+h) with bit h of e clear
 #pragma unroll
-          for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if ((e & h) == 0) {
-                const float a = v[e], b = v[e + h];
-                v[e] = __fadd_rn(a, b);
-                v[e + h] = __fsub_rn(a, b);
-              }
-            }
-          }
-          // butterflies across the L lanes of the group: stride 32m pairs lane j
-          // (bit m clear) with lane j^m; one exact FFMA per element: lower lane
-          // v + o, upper lane o - v (+-1 * v is exact)
-#pragma unroll
-          for (int m = 1; m < L; m <<= 1) {
-            const float sgn = (lq & m) ? -1.0f : 1.0f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __fmaf_rn(sgn, v[e], __shfl_xor_sync(gmask, v[e], m));
-          }
-          float amax = 0.f;
+        for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            v[e] = __fmul_rn(v[e], p.inv_sqrt_b);
-            amax = fmaxf(amax, fabsf(v[e]));
-          }
-          if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-            // perfect pairwise tree: five in-lane levels, then lanes by xor 1, 2, ..
-            float sq[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sq[e] = __fmul_rn(v[e], v[e]);
-#pragma unroll
-            for (int w = 1; w < 32; w <<= 1) {
-#pragma unroll
-              for (int e = 0; e < 32; e += 2 * w) sq[e] = __fadd_rn(sq[e], sq[e + w]);
+            if ((e & h) == 0) {
+              const float a = v[e], b = v[e + h];
+              v[e] = __fadd_rn(a, b);
+              v[e + h] = __fsub_rn(a, b);
             }
-            float ss = sq[0];
-#pragma unroll
-            for (int m = 1; m < L; m <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(gmask, ss, m));
-            if (lq == 0) part_ss[ri * nblk + bk] = ss;
-          } else if constexpr (WEIGHT && FMT == RQ_FMT_INT4) {
-            // one scale per 128 rotated coordinates = 4 lanes
-#pragma unroll
-            for (int m = 1; m < (L < 4 ? L : 4); m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
-            if ((lq & 3) == 0) atomicMax(&amax_bits[ri * ngrp + i0 / 128], __float_as_uint(amax));
-          } else {
-#pragma unroll
-            for (int m = 1; m < L; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
-            if (lq == 0) atomicMax(&amax_bits[ri], __float_as_uint(amax));
           }
         }
-      }
-      __syncthreads();
-      // the previous sub-group's amax words are free again (its quantization
-      // finished before the barrier above)
-      for (int i = threadIdx.x; i < Rs * ngrp; i += K1_THREADS)
-        amax_bits2[(size_t)((sg & 1) ^ 1) * Rs * ngrp + i] = 0u;
-      if constexpr (PROJ && !RESID) {
-        // weight rows were gathered straight from the row buffer: free now
-        if (s == nsub - 1 && threadIdx.x == 0 && has_next) {
-          fence_proxy_async_smem();
-          issue_group(g + gridDim.x, 0);
+        // butterflies across the L lanes of the group: stride 32m pairs lane j
+        // (bit m clear) with lane j^m; one exact FFMA per element: lower lane
+        // v + o, upper lane o - v (+-1 * v is exact)
+#pragma unroll
+        for (int m = 1; m < L; m <<= 1) {
+          const float sgn = (lq & m) ? -1.0f : 1.0f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __fmaf_rn(sgn, v[e], __shfl_xor_sync(gmask, v[e], m));
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          v[e] = __fmul_rn(v[e], p.inv_sqrt_b);
+          amax = fmaxf(amax, fabsf(v[e]));
+        }
+        if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+          // perfect pairwise tree: five in-lane levels, then lanes by xor 1, 2, ..
+          float sq[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sq[e] = __fmul_rn(v[e], v[e]);
+#pragma unroll
+          for (int w = 1; w < 32; w <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2 * w) sq[e] = __fadd_rn(sq[e], sq[e + w]);
+          }
+          float ss = sq[0];
+#pragma unroll
+          for (int m = 1; m < L; m <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(gmask, ss, m));
+          red[s] = ss;
+          if constexpr (IPW == 1) publish(ri, bk, ss);
+        } else if constexpr (WEIGHT && FMT == RQ_FMT_INT4) {
+          // one scale per 128 rotated coordinates = 4 lanes
+#pragma unroll
+          for (int m = 1; m < (L < 4 ? L : 4); m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
+          red[s] = amax;
+          if constexpr (IPW == 1) publish(ri, bk, amax);
+        } else {
+#pragma unroll
+          for (int m = 1; m < L; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, m));
+          red[s] = amax;
+          if constexpr (IPW == 1) publish(ri, bk, amax);
         }
       }
+    }
+    if constexpr (IPW > 1) {
+#pragma unroll
+      for (int s = 0; s < IPW; ++s) {
+        const int item = slot0 + s * SLOTS;
+        if (item < nitems) publish(item / nblk, item % nblk, red[s]);
+      }
+    }
+    __syncthreads();
+    if constexpr (PROJ) {
+      // the row buffer is free: stream the next group in behind the quantization
+      if (threadIdx.x == 0 && has_next) {
+        fence_proxy_async_smem();
+        issue_group(g + gridDim.x, 0);
+      }
+    }
+    // the other parity's amax words are free again (the previous group's
+    // quantization finished before the barrier above)
+    for (int i = threadIdx.x; i < R * ngrp; i += K1_THREADS) amax_bits2[(size_t)((it & 1) ^ 1) * R * ngrp + i] = 0u;
 
-      // ---------------------------------------------------------- phase B
+    // ------------------------------------------------------------ phase B
 #pragma unroll
-      for (int sl = 0; sl < IPW; ++sl) {
-        const int item = slot0 + sl * SLOTS;
-        if (item < nitems) {
-          const int ri = item / nblk, bk = item - ri * nblk;
-          const int row = r0 + rs0 + ri;
-          const int i0 = bk * B + lq * 32;
-          const float* v = y[sl];
-          uint32_t pk[4] = {0u, 0u, 0u, 0u};   // 32 codes, nibble e at bits 4(e%8) of word e/8
-          // row (or group) scale, derived by every lane from the block partials;
-          // the first lane of the row's (group's) first block writes it out
-          float mlt;
-          if constexpr (FMT == RQ_FMT_INT4) {
-            const float amax = __uint_as_float(amax_bits[ri * ngrp + (WEIGHT ? i0 / 128 : 0)]);
-            mlt = amax > 0.f ? __fdiv_rn(7.0f, amax) : 0.f;
-            if (WEIGHT ? (i0 % 128 == 0) : (bk == 0 && lq == 0)) {
-              const float sc = amax > 0.f ? __fdiv_rn(amax, 7.0f) : 0.f;
-              if constexpr (WEIGHT) p.scale[(size_t)(i0 / 128) * p.rows + row] = sc;
-              else p.scale[row] = sc;
-            }
-          } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-            float ss = part_ss[ri * nblk];
-            for (int j = 1; j < nblk; ++j) ss = __fadd_rn(ss, part_ss[ri * nblk + j]);
-            const float nrm = __fsqrt_rn(ss);
-            mlt = nrm > 0.f ? __fdiv_rn(p.sqrtK, nrm) : 0.f;
-            if (bk == 0 && lq == 0) p.scale[row] = nrm > 0.f ? __fdiv_rn(nrm, p.sqrtK) : 0.f;
-          } else {
-            const float amax = __uint_as_float(amax_bits[ri]);
-            mlt = amax > 0.f ? __fdiv_rn(2688.0f, amax) : 0.f;
-            if (bk == 0 && lq == 0) p.scale[row] = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 0.f;
+    for (int s = 0; s < IPW; ++s) {
+      const int item = slot0 + s * SLOTS;
+      if (item < nitems) {
+        const int ri = item / nblk, bk = item - ri * nblk;
+        const int row = r0 + ri;
+        const int i0 = bk * B + lq * 32;
+        const float* v = y[s];
+        uint32_t pk[4] = {0u, 0u, 0u, 0u};   // 32 codes, nibble e at bits 4(e%8) of word e/8
+        // row (or group) scale, derived by every lane from the block partials;
+        // the first lane of the row's (group's) first block writes it out
+        float mlt;
+        if constexpr (FMT == RQ_FMT_INT4) {
+          const float amax = __uint_as_float(amax_bits[ri * ngrp + (WEIGHT ? i0 / 128 : 0)]);
+          mlt = amax > 0.f ? __fdiv_rn(7.0f, amax) : 0.f;
+          if (WEIGHT ? (i0 % 128 == 0) : (bk == 0 && lq == 0)) {
+            const float sc = amax > 0.f ? __fdiv_rn(amax, 7.0f) : 0.f;
+            if constexpr (WEIGHT) p.scale[(size_t)(i0 / 128) * p.rows + row] = sc;
+            else p.scale[row] = sc;
           }
-          if constexpr (FMT == RQ_FMT_INT4) {
-            const float inv = mlt;
+        } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+          float ss = part_ss[ri * nblk];
+          for (int j = 1; j < nblk; ++j) ss = __fadd_rn(ss, part_ss[ri * nblk + j]);
+          const float nrm = __fsqrt_rn(ss);
+          mlt = nrm > 0.f ? __fdiv_rn(p.sqrtK, nrm) : 0.f;
+          if (bk == 0 && lq == 0) p.scale[row] = nrm > 0.f ? __fdiv_rn(nrm, p.sqrtK) : 0.f;
+        } else {
+          const float amax = __uint_as_float(amax_bits[ri]);
+          mlt = amax > 0.f ? __fdiv_rn(2688.0f, amax) : 0.f;
+          if (bk == 0 && lq == 0) p.scale[row] = amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 0.f;
+        }
+        if constexpr (FMT == RQ_FMT_INT4) {
+          const float inv = mlt;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              int q = __float2int_rn(__fmul_rn(v[e], inv));
-              q = max(-7, min(7, q));
-              pk[e >> 3] |= ((uint32_t)q & 0xFu) << (4 * (e & 7));
-            }
-          } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-            const float inv = mlt;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float u = __fmul_rn(v[e], inv);
-              // number of boundaries <= u (ascending, padded with +inf to 16)
-              uint32_t c = 0;
-              if constexpr (FMT == RQ_FMT_LM16) {
-#pragma unroll
-                for (int step = 8; step >= 1; step >>= 1)
-                  if (u >= bnd_s[c + step - 1]) c += step;
-                pk[e >> 3] |= c << (4 * (e & 7));
-              } else {
-                c = (u >= bnd_s[0]) + (u >= bnd_s[1]) + (u >= bnd_s[2]);
-                pk[e >> 4] |= c << (2 * (e & 15));
-              }
-            }
-          } else {  // NVFP4: two 16-element groups per lane
-            const float inv_t = mlt;
-            uint16_t sbs = 0;
-#pragma unroll
-            for (int gq = 0; gq < 2; ++gq) {
-              float u[16];
-              float m16 = 0.f;
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                u[e] = __fmul_rn(v[16 * gq + e], inv_t);
-                m16 = fmaxf(m16, fabsf(u[e]));
-              }
-              const float sbf = __fdiv_rn(m16, 6.0f);
-              const uint8_t sb = (uint8_t)(cvt_e4m3x2(0.f, sbf) & 0xFF);
-              const float rcp = sb ? __fdiv_rn(1.0f, e4m3_to_f32(sb)) : 0.f;
-#pragma unroll
-              for (int e = 0; e < 16; e += 2) {
-                const uint32_t byte = sb ? (uint32_t)cvt_e2m1x2(__fmul_rn(u[e + 1], rcp), __fmul_rn(u[e], rcp)) : 0u;
-                const int ee = 16 * gq + e;
-                pk[ee >> 3] |= byte << (4 * (ee & 7));
-              }
-              sbs |= (uint16_t)sb << (8 * gq);
-            }
-            // block scales kb, kb+1 (kb even) are adjacent bytes of the tile layout
-            *reinterpret_cast<uint16_t*>(p.bscale + sf_offset(row, i0 / 16, K)) = sbs;
+          for (int e = 0; e < 32; ++e) {
+            int q = __float2int_rn(__fmul_rn(v[e], inv));
+            q = max(-7, min(7, q));
+            pk[e >> 3] |= ((uint32_t)q & 0xFu) << (4 * (e & 7));
           }
-          if constexpr (FMT == RQ_FMT_LM4) {
-            *reinterpret_cast<uint2*>(p.codes + (size_t)row * (K / 4) + i0 / 4) = make_uint2(pk[0], pk[1]);
-          } else {
-            *reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 2) + i0 / 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+          const float inv = mlt;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float u = __fmul_rn(v[e], inv);
+            // number of boundaries <= u (ascending, padded with +inf to 16)
+            uint32_t c = 0;
+            if constexpr (FMT == RQ_FMT_LM16) {
+#pragma unroll
+              for (int step = 8; step >= 1; step >>= 1)
+                if (u >= bnd_s[c + step - 1]) c += step;
+              pk[e >> 3] |= c << (4 * (e & 7));
+            } else {
+              c = (u >= bnd_s[0]) + (u >= bnd_s[1]) + (u >= bnd_s[2]);
+              pk[e >> 4] |= c << (2 * (e & 15));
+            }
           }
+        } else {  // NVFP4: two 16-element groups per lane
+          const float inv_t = mlt;
+          uint16_t sbs = 0;
+#pragma unroll
+          for (int gq = 0; gq < 2; ++gq) {
+            float u[16];
+            float m16 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              u[e] = __fmul_rn(v[16 * gq + e], inv_t);
+              m16 = fmaxf(m16, fabsf(u[e]));
+            }
+            const float sbf = __fdiv_rn(m16, 6.0f);
+            const uint8_t sb = (uint8_t)(cvt_e4m3x2(0.f, sbf) & 0xFF);
+            const float rcp = sb ? __fdiv_rn(1.0f, e4m3_to_f32(sb)) : 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const uint32_t byte = sb ? (uint32_t)cvt_e2m1x2(__fmul_rn(u[e + 1], rcp), __fmul_rn(u[e], rcp)) : 0u;
+              const int ee = 16 * gq + e;
+              pk[ee >> 3] |= byte << (4 * (ee & 7));
+            }
+            sbs |= (uint16_t)sb << (8 * gq);
+          }
+          // block scales kb, kb+1 (kb even) are adjacent bytes of the tile layout
+          *reinterpret_cast<uint16_t*>(p.bscale + sf_offset(row, i0 / 16, K)) = sbs;
+        }
+        if constexpr (FMT == RQ_FMT_LM4) {
+          *reinterpret_cast<uint2*>(p.codes + (size_t)row * (K / 4) + i0 / 4) = make_uint2(pk[0], pk[1]);
+        } else {
+          *reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 2) + i0 / 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
     }
   }
 }
 
-size_t k1_smem_bytes(int R, int Rs, int K, int nblk, bool proj, bool resid, int ngrp) {
-  size_t off = (size_t)(proj ? 1 : 2) * R * K * 2;
-  if (resid) off += (size_t)Rs * K * 4;
-  if (proj) off += (size_t)32 * ut_pitch(K) * 2 + (size_t)R * 32 * 2;
-  off += (size_t)2 * Rs * nblk * 4;
-  off += (size_t)2 * Rs * ngrp * 4;
+
+size_t k1_smem_bytes(int R, int K, int nblk, bool proj, int ngrp) {
+  size_t off = proj ? (size_t)R * K * 4 + (size_t)32 * ut_pitch(K) * 2 + (size_t)R * 32 * 4 + (size_t)K * 4
+                    : (size_t)2 * R * K * 2;
+  off += (size_t)2 * R * nblk * 4;
+  off += (size_t)2 * R * ngrp * 4;
   off = (off + 15) & ~(size_t)15;
   return off + 32 + 64;
 }
@@ -509,45 +585,22 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
   const int nblk = a.K / (L * 32);
   const int ngrp = (WEIGHT && FMT == RQ_FMT_INT4) ? a.K / 128 : 1;
   const int sms = a.num_sms > 0 ? a.num_sms : 148;
-  int R = 0, Rs = 0;
-  size_t smem = 0;
-  if constexpr (PROJ) {
-    // one load of R rows per CTA and wave (at most 32: two coefficient chains
-    // per thread), rotated in sub-groups of at most 16 rows that fit the slots
-    const size_t cap = 232448;
-    int R0 = (a.rows + sms - 1) / sms;
-    R0 = R0 < 1 ? 1 : (R0 > 32 ? 32 : R0);
-    for (int r = R0; r >= 1 && !R; --r) {
-      for (int nsub = (r + 15) / 16; nsub <= r; ++nsub) {
-        const int rs = (r + nsub - 1) / nsub;
-        if (rs * nblk > SLOTS * IPW) continue;
-        const size_t b = k1_smem_bytes(r, rs, a.K, nblk, true, !WEIGHT, ngrp);
-        if (b <= cap) {
-          R = r;
-          Rs = rs;
-          smem = b;
-          break;
-        }
-      }
-    }
-    if (!R) return cudaErrorInvalidValue;
-  } else {
-    // rows per group: as many as fill IPW passes of the block slots
-    R = (SLOTS * IPW) / nblk;
-    if (R < 1) return cudaErrorInvalidValue;
-    if (R > 24) R = 24;
-    smem = k1_smem_bytes(R, R, a.K, nblk, false, false, ngrp);
-    // two CTAs per SM for the single-pass variant
-    const size_t cap = IPW == 1 ? 110 * 1024 : 200 * 1024;
-    while (smem > cap && R > 1) {
-      --R;
-      smem = k1_smem_bytes(R, R, a.K, nblk, false, false, ngrp);
-    }
-    if (smem > cap) return cudaErrorInvalidValue;
-    Rs = R;
+  // rows per group: as many as fill IPW passes of the block slots; with the
+  // projection no more than one wave needs (every SM busy with the chains)
+  int R = (SLOTS * IPW) / nblk;
+  if (R < 1) return cudaErrorInvalidValue;
+  if (R > 24 && !PROJ) R = 24;
+  // (the coefficient and residual mappings cover at most 32 rows)
+  if (PROJ) R = min(min(R, 32), max(1, (a.rows + sms - 1) / sms));
+  size_t smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp);
+  // two CTAs per SM for the single-pass variant
+  const size_t cap = PROJ ? 232448 : IPW == 1 ? 110 * 1024 : 200 * 1024;
+  while (smem > cap && R > 1) {
+    --R;
+    smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp);
   }
+  if (smem > cap) return cudaErrorInvalidValue;
   p.R = R;
-  p.Rs = Rs;
   p.ngroups = (a.rows + R - 1) / R;
   auto kern = k1_rotate_quantize<L, FMT, PROJ, WEIGHT, IPW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
