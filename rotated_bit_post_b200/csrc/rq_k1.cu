@@ -28,7 +28,9 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
+#include <cstring>
 
 #include "rq_internal.h"
 #include "rq_ptx.cuh"
@@ -38,6 +40,7 @@ namespace rq {
 namespace {
 
 constexpr int K1_THREADS = 512;
+constexpr int K1_LUT_MAX = 512;
 constexpr int K1_WARPS = K1_THREADS / 32;
 
 struct __align__(16) K1Params {
@@ -56,6 +59,12 @@ struct __align__(16) K1Params {
   float sqrtK;             // fp32(sqrt(K))
   int32_t nbnd;            // number of codebook boundaries (levels - 1)
   float bnd[15];
+  // codebook search table: u * 2^lut_shift, clamped to [lut_gmin, lut_gmin +
+  // lut_n - 1] and floored, indexes cells of width 2^-lut_shift holding at most
+  // one boundary each: code = lut[g].x + (u >= lut[g].y as float)
+  int32_t lut_shift, lut_gmin, lut_n;
+  uint2 lut[K1_LUT_MAX];
+  float rcp_e4m3[128];     // fp32(1 / e4m3 value) for the positive e4m3 codes, 0 for code 0
 };
 
 
@@ -78,6 +87,39 @@ __device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float acc) {
       : "=f"(d)
       : "r"(a), "r"(b), "f"(acc), "n"(AH), "n"(BH));
   return d;
+}
+
+// Packed FP32 pairs (sm_100 f32x2 arithmetic): each lane rounds exactly like
+// the scalar instruction, two elements per issue slot.
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+// (a, b) -> (a + b, a - b) for the element pairs (a0, b0) and (a1, b1)
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
+  asm("{\n\t.reg .b64 a, b, s, d;\n\t"
+      "mov.b64 a, {%0, %1};\n\tmov.b64 b, {%2, %3};\n\t"
+      "add.rn.f32x2 s, a, b;\n\tsub.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, s;\n\tmov.b64 {%2, %3}, d;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+// v = s * v + o on two elements, s a packed pair
+__device__ __forceinline__ void fma2(float& v0, float& v1, uint64_t s2, float o0, float o1) {
+  asm("{\n\t.reg .b64 v, o;\n\t"
+      "mov.b64 v, {%0, %1};\n\tmov.b64 o, {%3, %4};\n\t"
+      "fma.rn.f32x2 v, %2, v, o;\n\tmov.b64 {%0, %1}, v;\n\t}"
+      : "+f"(v0), "+f"(v1) : "l"(s2), "f"(o0), "f"(o1));
+}
+// v = v * s on two elements, s a packed pair
+__device__ __forceinline__ void mul2(float& v0, float& v1, uint64_t s2) {
+  asm("{\n\t.reg .b64 v;\n\tmov.b64 v, {%0, %1};\n\tmul.rn.f32x2 v, v, %2;\n\tmov.b64 {%0, %1}, v;\n\t}"
+      : "+f"(v0), "+f"(v1) : "l"(s2));
+}
+// round to the nearest integer, ties to even, for |x| < 2^22 (full-rate FP32
+// add in place of a conversion)
+__device__ __forceinline__ int rint_small(float x) {
+  return __float_as_int(__fadd_rn(x, 12582912.0f)) - 0x4B400000;
 }
 
 // Projection layout in shared memory: U^T as BF16 rows of KP = K + 8 entries
@@ -106,10 +148,10 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
   //   without projection: [2][R][K] bf16 row buffers (the next group streams in
   //   while this one is transformed)
   //   with projection: [R][K] fp32 rows (the bf16 rows land in its upper half
-  //   and are widened in place) | [32][K+8] bf16 U^T | [R][32] fp32 -c |
-  //   [K] int32 signed permutation
-  //   then [2][R][nblk] fp32 block sum-of-squares | [2][R][ngrp] u32 amax bits |
-  //   mbarriers | abort flag | boundaries
+  //   and are widened in place) | [32][K+8] bf16 U^T | [R][32] fp32 -c
+  //   then [K] int32 signed permutation | [2][R][nblk] fp32 block sum-of-squares |
+  //   [2][R][ngrp] u32 amax bits | mbarriers | abort flag | boundaries |
+  //   [128] fp32 e4m3 reciprocals | [lut_n] codebook search cells
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
   float* xf = reinterpret_cast<float*>(smem);
   uint16_t* land = reinterpret_cast<uint16_t*>(smem + (PROJ ? (size_t)R * K * 2 : 0));
@@ -123,11 +165,11 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     off += (size_t)32 * ut_pitch(K) * 2;
     negc = reinterpret_cast<float*>(smem + off);
     off += (size_t)R * 32 * 4;
-    rot_s = reinterpret_cast<int32_t*>(smem + off);
-    off += (size_t)K * 4;
   } else {
     off = (size_t)2 * R * K * 2;
   }
+  rot_s = reinterpret_cast<int32_t*>(smem + off);
+  off += (size_t)K * 4;
   // block partials, double-buffered by group parity so that no barrier is
   // needed between a group's quantization and the next group's reductions
   float* part_ss2 = reinterpret_cast<float*>(smem + off);
@@ -138,8 +180,12 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
   off = (off + 15) & ~(size_t)15;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + off + 16);
-  float* bnd_s = reinterpret_cast<float*>(smem + off + 32);  // 16 codebook boundaries
-  if (threadIdx.x < 16) bnd_s[threadIdx.x] = threadIdx.x < p.nbnd ? p.bnd[threadIdx.x] : __int_as_float(0x7f800000);
+  float* rcp_s = reinterpret_cast<float*>(smem + off + 96);
+  uint2* lut_s = reinterpret_cast<uint2*>(smem + off + 96 + 512);
+  if constexpr (FMT == RQ_FMT_NVFP4)
+    for (int i = threadIdx.x; i < 128; i += K1_THREADS) rcp_s[i] = p.rcp_e4m3[i];
+  if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4)
+    for (int i = threadIdx.x; i < p.lut_n; i += K1_THREADS) lut_s[i] = p.lut[i];
 
   const uint32_t row_bytes = (uint32_t)K * 2;
 
@@ -175,9 +221,9 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
         ut[(size_t)(8 * q + 2 * h + 1) * KP + k] = (uint16_t)(ww[h] >> 16);
       }
     }
-    for (int t = threadIdx.x; t < K / 4; t += K1_THREADS)
-      reinterpret_cast<int4*>(rot_s)[t] = __ldg(reinterpret_cast<const int4*>(p.rot) + t);
   }
+  for (int t = threadIdx.x; t < K / 4; t += K1_THREADS)
+    reinterpret_cast<int4*>(rot_s)[t] = __ldg(reinterpret_cast<const int4*>(p.rot) + t);
 
   for (int i = threadIdx.x; i < 2 * R * ngrp; i += K1_THREADS) amax_bits2[i] = 0u;
   int it = 0;
@@ -371,10 +417,10 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
         const int ri = item / nblk, bk = item - ri * nblk;
         const int i0 = bk * B + lq * 32;
         float* v = y[s];
-        const int4* rp = reinterpret_cast<const int4*>((PROJ ? rot_s : p.rot) + i0);
+        const int4* rp = reinterpret_cast<const int4*>(rot_s + i0);
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
-          const int4 rv = PROJ ? rp[e4] : __ldg(rp + e4);
+          const int4 rv = rp[e4];
           const int rr[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -385,17 +431,19 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
             v[4 * e4 + q] = __uint_as_float(__float_as_uint(xv) ^ ((uint32_t)rr[q] & 0x80000000u));
           }
         }
-        // butterflies inside the lane: stride h pairs (e, e+h) with bit h of e clear
+        // butterflies inside the lane: stride h pairs (e, e+h) with bit h of e
+        // clear; from h = 2 on, the butterflies of e and e+1 share a packed op
 #pragma unroll
-        for (int h = 1; h < 32; h <<= 1) {
+        for (int e = 0; e < 32; e += 2) {
+          const float a = v[e], b = v[e + 1];
+          v[e] = __fadd_rn(a, b);
+          v[e + 1] = __fsub_rn(a, b);
+        }
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if ((e & h) == 0) {
-              const float a = v[e], b = v[e + h];
-              v[e] = __fadd_rn(a, b);
-              v[e + h] = __fsub_rn(a, b);
-            }
-          }
+        for (int h = 2; h < 32; h <<= 1) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            if ((e & h) == 0) bfly2(v[e], v[e + 1], v[e + h], v[e + h + 1]);
         }
         // butterflies across the L lanes of the group: stride 32m pairs lane j
         // (bit m clear) with lane j^m; one exact FFMA per element: lower lane
@@ -403,14 +451,19 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
 #pragma unroll
         for (int m = 1; m < L; m <<= 1) {
           const float sgn = (lq & m) ? -1.0f : 1.0f;
+          const uint64_t sgn2 = pack2(sgn, sgn);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __fmaf_rn(sgn, v[e], __shfl_xor_sync(gmask, v[e], m));
+          for (int e = 0; e < 32; e += 2) {
+            const float o0 = __shfl_xor_sync(gmask, v[e], m), o1 = __shfl_xor_sync(gmask, v[e + 1], m);
+            fma2(v[e], v[e + 1], sgn2, o0, o1);
+          }
         }
         float amax = 0.f;
+        const uint64_t isb2 = pack2(p.inv_sqrt_b, p.inv_sqrt_b);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          v[e] = __fmul_rn(v[e], p.inv_sqrt_b);
-          amax = fmaxf(amax, fabsf(v[e]));
+        for (int e = 0; e < 32; e += 2) {
+          mul2(v[e], v[e + 1], isb2);
+          amax = fmaxf(amax, fmaxf(fabsf(v[e]), fabsf(v[e + 1])));
         }
         if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
           // perfect pairwise tree: five in-lane levels, then lanes by xor 1, 2, ..
@@ -468,7 +521,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
         const int ri = item / nblk, bk = item - ri * nblk;
         const int row = r0 + ri;
         const int i0 = bk * B + lq * 32;
-        const float* v = y[s];
+        float* v = y[s];
         uint32_t pk[4] = {0u, 0u, 0u, 0u};   // 32 codes, nibble e at bits 4(e%8) of word e/8
         // row (or group) scale, derived by every lane from the block partials;
         // the first lane of the row's (group's) first block writes it out
@@ -482,8 +535,14 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
             else p.scale[row] = sc;
           }
         } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-          float ss = part_ss[ri * nblk];
-          for (int j = 1; j < nblk; ++j) ss = __fadd_rn(ss, part_ss[ri * nblk + j]);
+          // the row's sum of squares, block by block in order: the group's
+          // first lane adds, the others take its result
+          float ss = 0.f;
+          if (lq == 0) {
+            ss = part_ss[ri * nblk];
+            for (int j = 1; j < nblk; ++j) ss = __fadd_rn(ss, part_ss[ri * nblk + j]);
+          }
+          ss = __shfl_sync(gmask, ss, lane & ~(L - 1));
           const float nrm = __fsqrt_rn(ss);
           mlt = nrm > 0.f ? __fdiv_rn(p.sqrtK, nrm) : 0.f;
           if (bk == 0 && lq == 0) p.scale[row] = nrm > 0.f ? __fdiv_rn(nrm, p.sqrtK) : 0.f;
@@ -496,42 +555,43 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
           const float inv = mlt;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            int q = __float2int_rn(__fmul_rn(v[e], inv));
+            int q = rint_small(__fmul_rn(v[e], inv));   // |v * inv| <= 7 (+ rounding)
             q = max(-7, min(7, q));
             pk[e >> 3] |= ((uint32_t)q & 0xFu) << (4 * (e & 7));
           }
         } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+          // code = number of boundaries <= u, read from the cell of u: its
+          // base count plus one compare against the cell's boundary (if any)
           const float inv = mlt;
+          const float cscale = __int_as_float((127 + p.lut_shift) << 23);   // 2^lut_shift
+          const float tlo = (float)p.lut_gmin, thi = (float)(p.lut_gmin + p.lut_n - 1) + 0.5f;
+          const int gbias = 0x4B400000 + p.lut_gmin;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float u = __fmul_rn(v[e], inv);
-            // number of boundaries <= u (ascending, padded with +inf to 16)
-            uint32_t c = 0;
-            if constexpr (FMT == RQ_FMT_LM16) {
-#pragma unroll
-              for (int step = 8; step >= 1; step >>= 1)
-                if (u >= bnd_s[c + step - 1]) c += step;
-              pk[e >> 3] |= c << (4 * (e & 7));
-            } else {
-              c = (u >= bnd_s[0]) + (u >= bnd_s[1]) + (u >= bnd_s[2]);
-              pk[e >> 4] |= c << (2 * (e & 15));
-            }
+            const float t = fminf(fmaxf(__fmul_rn(u, cscale), tlo), thi);   // exact scaling
+            const int g = __float_as_int(__fadd_rd(t, 12582912.0f)) - gbias;  // floor(t) - gmin
+            const uint2 cell = lut_s[g];
+            const uint32_t c = cell.x + (u >= __uint_as_float(cell.y) ? 1u : 0u);
+            if constexpr (FMT == RQ_FMT_LM16) pk[e >> 3] |= c << (4 * (e & 7));
+            else pk[e >> 4] |= c << (2 * (e & 15));
           }
         } else {  // NVFP4: two 16-element groups per lane
           const float inv_t = mlt;
           uint16_t sbs = 0;
 #pragma unroll
           for (int gq = 0; gq < 2; ++gq) {
-            float u[16];
+            float* u = v + 16 * gq;   // scaled in place
             float m16 = 0.f;
+            const uint64_t it2 = pack2(inv_t, inv_t);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              u[e] = __fmul_rn(v[16 * gq + e], inv_t);
-              m16 = fmaxf(m16, fabsf(u[e]));
+            for (int e = 0; e < 16; e += 2) {
+              mul2(u[e], u[e + 1], it2);
+              m16 = fmaxf(m16, fmaxf(fabsf(u[e]), fabsf(u[e + 1])));
             }
             const float sbf = __fdiv_rn(m16, 6.0f);
             const uint8_t sb = (uint8_t)(cvt_e4m3x2(0.f, sbf) & 0xFF);
-            const float rcp = sb ? __fdiv_rn(1.0f, e4m3_to_f32(sb)) : 0.f;
+            const float rcp = rcp_s[sb & 0x7F];   // 1 / e4m3 value, 0 for code 0
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
               const uint32_t byte = sb ? (uint32_t)cvt_e2m1x2(__fmul_rn(u[e + 1], rcp), __fmul_rn(u[e], rcp)) : 0u;
@@ -554,13 +614,49 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
 }
 
 
-size_t k1_smem_bytes(int R, int K, int nblk, bool proj, int ngrp) {
-  size_t off = proj ? (size_t)R * K * 4 + (size_t)32 * ut_pitch(K) * 2 + (size_t)R * 32 * 4 + (size_t)K * 4
+size_t k1_smem_bytes(int R, int K, int nblk, bool proj, int ngrp, int lut_n) {
+  size_t off = proj ? (size_t)R * K * 4 + (size_t)32 * ut_pitch(K) * 2 + (size_t)R * 32 * 4
                     : (size_t)2 * R * K * 2;
+  off += (size_t)K * 4;
   off += (size_t)2 * R * nblk * 4;
   off += (size_t)2 * R * ngrp * 4;
   off = (off + 15) & ~(size_t)15;
-  return off + 32 + 64;
+  return off + 96 + 512 + (size_t)lut_n * 8;
+}
+
+// Host: e4m3 code (positive) -> value.
+float e4m3_value(int c) {
+  const int e = (c >> 3) & 15, m = c & 7;
+  return e == 0 ? std::ldexp((float)m, -9) : std::ldexp(1.0f + m / 8.0f, e - 7);
+}
+
+// Host: the codebook search table over cells of width 2^-shift, the coarsest
+// grid whose cells hold at most one boundary each.
+bool build_code_lut(K1Params& p, const float* bnd, int nbnd) {
+  for (int shift = 3; shift <= 14; ++shift) {
+    long cell[15];
+    bool ok = true;
+    for (int i = 0; i < nbnd; ++i) {
+      cell[i] = (long)std::floor(std::ldexp((double)bnd[i], shift));   // exact
+      if (i > 0 && cell[i] <= cell[i - 1]) ok = false;
+    }
+    if (!ok) continue;
+    const long gmin = cell[0] - 1, gmax = cell[nbnd - 1] + 1;
+    if (gmax - gmin + 1 > K1_LUT_MAX) return false;
+    p.lut_shift = shift;
+    p.lut_gmin = (int32_t)gmin;
+    p.lut_n = (int32_t)(gmax - gmin + 1);
+    for (long g = gmin; g <= gmax; ++g) {
+      uint32_t base = 0, b = 0x7f800000u;   // no boundary in the cell: +inf
+      for (int i = 0; i < nbnd; ++i) {
+        if (cell[i] < g) ++base;
+        if (cell[i] == g) std::memcpy(&b, &bnd[i], 4);
+      }
+      p.lut[g - gmin] = make_uint2(base, b);
+    }
+    return true;
+  }
+  return false;
 }
 
 template <int L, int FMT, bool PROJ, bool WEIGHT, int IPW>
@@ -582,6 +678,11 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
   p.sqrtK = a.sqrtK;
   p.nbnd = a.nbnd;
   for (int i = 0; i < 15; ++i) p.bnd[i] = i < a.nbnd ? a.bnd[i] : 0.f;
+  p.lut_n = 0;
+  if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
+    if (a.nbnd < 1 || !build_code_lut(p, a.bnd, a.nbnd)) return cudaErrorInvalidValue;
+  }
+  for (int c = 0; c < 128; ++c) p.rcp_e4m3[c] = (c == 0 || c == 0x7F) ? 0.f : 1.0f / e4m3_value(c);
   const int nblk = a.K / (L * 32);
   const int ngrp = (WEIGHT && FMT == RQ_FMT_INT4) ? a.K / 128 : 1;
   const int sms = a.num_sms > 0 ? a.num_sms : 148;
@@ -592,12 +693,12 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
   if (R > 24 && !PROJ) R = 24;
   // (the coefficient and residual mappings cover at most 32 rows)
   if (PROJ) R = min(min(R, 32), max(1, (a.rows + sms - 1) / sms));
-  size_t smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp);
+  size_t smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp, p.lut_n);
   // two CTAs per SM for the single-pass variant
   const size_t cap = PROJ ? 232448 : IPW == 1 ? 110 * 1024 : 200 * 1024;
   while (smem > cap && R > 1) {
     --R;
-    smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp);
+    smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp, p.lut_n);
   }
   if (smem > cap) return cudaErrorInvalidValue;
   p.R = R;
@@ -613,11 +714,15 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
 
 template <int L, int FMT, bool PROJ, bool WEIGHT>
 cudaError_t launch_k1_ipw(const K1Launch& a, cudaStream_t st) {
-  // single pass (two CTAs per SM) whenever one row fits in the block slots;
-  // the projection keeps one CTA per SM (its staged U fills shared memory)
+  // single pass (two CTAs per SM) whenever one row fits in the block slots and
+  // one row's buffers fit half of shared memory; the projection keeps one CTA
+  // per SM (its staged U fills shared memory)
   constexpr int SLOTS = K1_WARPS * (32 / L);
   if constexpr (!PROJ) {
-    if (SLOTS / (a.K / (L * 32)) >= 1) return launch_k1_t<L, FMT, PROJ, WEIGHT, 1>(a, st);
+    const int nblk = a.K / (L * 32);
+    const int ngrp = (WEIGHT && FMT == RQ_FMT_INT4) ? a.K / 128 : 1;
+    if (SLOTS / nblk >= 1 && k1_smem_bytes(1, a.K, nblk, false, ngrp, K1_LUT_MAX) <= 110 * 1024)
+      return launch_k1_t<L, FMT, PROJ, WEIGHT, 1>(a, st);
   }
   return launch_k1_t<L, FMT, PROJ, WEIGHT, 2>(a, st);
 }
