@@ -222,8 +222,14 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
       }
     }
   }
-  for (int t = threadIdx.x; t < K / 4; t += K1_THREADS)
-    reinterpret_cast<int4*>(rot_s)[t] = __ldg(reinterpret_cast<const int4*>(p.rot) + t);
+  // the signed permutation, interleaved per block so that the lanes of a group
+  // read consecutive 16-byte words: entry e of lane lq in block bk (rotated
+  // coordinate bk*B + 32*lq + e) sits at bk*B + (e/4)*4L + 4*lq + e%4
+  for (int t = threadIdx.x; t < K / 4; t += K1_THREADS) {
+    const int i = 4 * t, bk = i / B, w = i % B, l = w >> 5, e = w & 31;
+    reinterpret_cast<int4*>(rot_s)[(bk * B + (e >> 2) * 4 * L + 4 * l) >> 2] =
+        __ldg(reinterpret_cast<const int4*>(p.rot) + t);
+  }
 
   for (int i = threadIdx.x; i < 2 * R * ngrp; i += K1_THREADS) amax_bits2[i] = 0u;
   int it = 0;
@@ -417,10 +423,10 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
         const int ri = item / nblk, bk = item - ri * nblk;
         const int i0 = bk * B + lq * 32;
         float* v = y[s];
-        const int4* rp = reinterpret_cast<const int4*>(rot_s + i0);
+        const int4* rp = reinterpret_cast<const int4*>(rot_s + bk * B + 4 * lq);
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
-          const int4 rv = rp[e4];
+          const int4 rv = rp[e4 * L];
           const int rr[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
