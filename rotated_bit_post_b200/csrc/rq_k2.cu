@@ -273,20 +273,22 @@ struct Fp8Plan {
 // Threads: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, then the
 // epilogue warps from warp 4 (4 warps; 16 when GROUPED: four per TMEM lane
 // quadrant, each owning 32 of the 128 columns and their running sums) and the
-// code expansion warps: eight after the epilogue, or, when GROUPED, warps 2-3
-// plus two after the epilogue (704 threads, so that the 16 epilogue warps keep
-// their running sums in registers without spilling).
+// code expansion warps: sixteen after the epilogue for BN = 256 (eight for
+// BN = 128; the codebook lookups are issue-bound and four warps per scheduler
+// hide their latencies), or, when
+// GROUPED, warps 2-3 plus two after the epilogue (704 threads, so that the 16
+// epilogue warps keep their running sums in registers without spilling).
 // TMEM columns: GROUPED (INT4 weights, BN = 128): three per-group partials at
 // 0, 128, 256 (the running sum lives in the epilogue's registers), low-rank at
 // 384.  Otherwise: accumulators at 0 and BN (double-buffered across tiles),
 // low-rank at 384 when BN == 128.
-template <bool GROUPED>
-constexpr int fp8_threads() { return GROUPED ? 704 : 512; }
+template <int BN, bool GROUPED>
+constexpr int fp8_threads() { return GROUPED ? 704 : BN == 256 ? 768 : 512; }
 
 template <int BN, int WBITS, bool GROUPED>
-__global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
   using P = Fp8Plan<BN, WBITS>;
-  constexpr int NW = fp8_threads<GROUPED>() / 32;
+  constexpr int NW = fp8_threads<BN, GROUPED>() / 32;
   constexpr int NEPI = GROUPED ? 16 : 4;         // epilogue warps
   constexpr int EXP0 = 4 + NEPI;                 // first expansion warp
   constexpr int NXW = GROUPED ? 4 : NW - EXP0;   // expansion warps
@@ -599,16 +601,18 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
         }
         // A: 128 rows x 4 segments of 16 packed bytes (32 codes); 8 consecutive
         // threads take 8 consecutive rows of one segment (conflict-free both ways)
-        uint4 va[512 / NXT];
+        constexpr int NA = (512 + NXT - 1) / NXT;
+        uint4 va[NA];
 #pragma unroll
-        for (int it = 0; it < 512 / NXT; ++it) {
+        for (int it = 0; it < NA; ++it) {
           const int idx = it * NXT + t;
           const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-          va[it] = ld_shared_v4(pa + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+          if (idx < 512) va[it] = ld_shared_v4(pa + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
         }
 #pragma unroll
-        for (int it = 0; it < 512 / NXT; ++it) {
+        for (int it = 0; it < NA; ++it) {
           const int idx = it * NXT + t;
+          if (idx >= 512) break;
           const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
           const uint4 v = va[it];
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -620,16 +624,18 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
           st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
         }
         if constexpr (WBITS == 4) {
-          uint4 vb[BN * 4 / NXT];
+          constexpr int NBI = (BN * 4 + NXT - 1) / NXT;
+          uint4 vb[NBI];
 #pragma unroll
-          for (int it = 0; it < BN * 4 / NXT; ++it) {
+          for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
             const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-            vb[it] = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+            if (idx < BN * 4) vb[it] = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
           }
 #pragma unroll
-          for (int it = 0; it < BN * 4 / NXT; ++it) {
+          for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
+            if (idx >= BN * 4) break;
             const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
             const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -642,16 +648,18 @@ __global__ void __launch_bounds__(fp8_threads<GROUPED>(), 1) gemm_fp8_kernel(con
           }
         } else {
           // 2-bit weights: 32 packed bytes per row = 2 segments of 64 codes
-          uint4 vb[BN * 2 / NXT];
+          constexpr int NBI = (BN * 2 + NXT - 1) / NXT;
+          uint4 vb[NBI];
 #pragma unroll
-          for (int it = 0; it < BN * 2 / NXT; ++it) {
+          for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
             const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
-            vb[it] = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
+            if (idx < BN * 2) vb[it] = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
           }
 #pragma unroll
-          for (int it = 0; it < BN * 2 / NXT; ++it) {
+          for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
+            if (idx >= BN * 2) break;
             const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
             const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -991,13 +999,13 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 2, a.N, a.K / 2, 64, BN,
                       CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) { *why = "cuTensorMapEncodeTiled failed"; return cudaErrorInvalidValue; }
-  if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<true>(), tm, gp, st);
+  if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<128, true>(), tm, gp, st);
   if (BN == 256) {
-    if (w2) return launch(gemm_fp8_kernel<256, 2, false>, Fp8Plan<256, 2>::BYTES, grid, 512, tm, gp, st);
-    return launch(gemm_fp8_kernel<256, 4, false>, Fp8Plan<256, 4>::BYTES, grid, 512, tm, gp, st);
+    if (w2) return launch(gemm_fp8_kernel<256, 2, false>, Fp8Plan<256, 2>::BYTES, grid, fp8_threads<256, false>(), tm, gp, st);
+    return launch(gemm_fp8_kernel<256, 4, false>, Fp8Plan<256, 4>::BYTES, grid, fp8_threads<256, false>(), tm, gp, st);
   }
-  if (w2) return launch(gemm_fp8_kernel<128, 2, false>, Fp8Plan<128, 2>::BYTES, grid, 512, tm, gp, st);
-  return launch(gemm_fp8_kernel<128, 4, false>, Fp8Plan<128, 4>::BYTES, grid, 512, tm, gp, st);
+  if (w2) return launch(gemm_fp8_kernel<128, 2, false>, Fp8Plan<128, 2>::BYTES, grid, fp8_threads<128, false>(), tm, gp, st);
+  return launch(gemm_fp8_kernel<128, 4, false>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<128, false>(), tm, gp, st);
 }
 
 }  // namespace rq
