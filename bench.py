@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-bf16-linear", action="store_true", help="skip the cuBLAS BF16 linear on the same shapes")
     return ap.parse_args()
 
 
@@ -289,6 +290,28 @@ def run_ours(args, w, rank, world, dist):
     if rc != 0:
         raise RuntimeError(f"kernel status {code:#x}")
 
+    # ---------------- the same layer as a plain BF16 linear (cuBLAS via torch), for context
+    bf16_linear = None
+    if not args.no_bf16_linear:
+        Wb = torch.from_numpy(inputs.weights(w).view(np.int16)).to(dev).view(torch.bfloat16)
+        Xb = X.view(torch.bfloat16)
+        Yb = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            torch.matmul(Xb, Wb.t(), out=Yb)
+        n_lin = max(5, min(50, args.steps))
+        evl = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_lin)]
+        for a, b in evl:
+            flush.zero_()
+            a.record(stream)
+            torch.matmul(Xb, Wb.t(), out=Yb)
+            b.record(stream)
+        torch.cuda.synchronize()
+        lin_ms = statistics.mean(a.elapsed_time(b) for a, b in evl)
+        bf16_linear = {"ms": lin_ms, "tflops": 2.0 * w.M * w.N * w.K / (lin_ms * 1e-3) / 1e12,
+                       "tokens_per_s": w.M / (lin_ms * 1e-3), "what": "torch.matmul BF16 x BF16^T (cuBLAS), "
+                       "same M, N, K, L2 flushed before each call, no rotation or quantization"}
+        del Wb, Yb
+
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -357,15 +380,19 @@ def run_ours(args, w, rank, world, dist):
                        "k1_frac_hbm": k1_gbs / pk["hbm_gbs"], "k2_gemm_us": 1e3 * k2_ms,
                        "k2_tflops": k2_tflops, "k2_frac_peak": k2_tflops / tensor_peak},
            "roofline": roof, "clocks": clocks.summary(), "e2e": e2e,
+           "bf16_linear": bf16_linear,
+           "speedup_vs_bf16_linear": None if bf16_linear is None else bf16_linear["ms"] / ms_per_step,
            "gpu_launches": 2 * args.steps}
     if not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(out), flush=True)
 
 
-# DRAM bytes per launch of the GEMM from ncu (read + write), keyed by workload;
-# filled in from profiles/ when a capture of the current kernel exists.
-TRAFFIC = {}
+# DRAM bytes per launch of the GEMM (read + write) from a 1-pass ncu capture of
+# the current kernels at the full sizes, keyed by workload (see
+# profiles/dram_traffic_all_workloads.md).
+TRAFFIC = {"c2": 5_790_720 + 37_376, "c3": 21_344_768 + 32_366_848, "c4": 53_147_904 + 3_260_672,
+           "c5": 54_207_232 + 1_119_752_960}
 
 
 def main():
