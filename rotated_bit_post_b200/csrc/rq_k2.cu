@@ -52,6 +52,7 @@ struct __align__(64) TMaps {
   CUtensorMap b;   // packed weight codes
   CUtensorMap c;   // low-rank coefficients (M x r BF16)
   CUtensorMap l;   // low-rank weights (N x r BF16)
+  CUtensorMap y;   // BF16 output, 32 x 32 boxes, 64-byte swizzle (TMA-store epilogue)
 };
 
 struct __align__(16) GemmParams {
@@ -66,6 +67,7 @@ struct __align__(16) GemmParams {
   int has_lr;
   void* Y;
   int out_fp32;
+  int tma_store;           // BF16 output written through shared memory + TMA stores
   int32_t* status;
 };
 
@@ -76,14 +78,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Four 4-bit codes (bits 0-15 of x) -> four LUT bytes.
-__device__ __forceinline__ uint32_t lut16x4(uint32_t x, const uint32_t (&L)[4]) {
-  const uint32_t sel = x & 0x7777u;
-  const uint32_t lo = prmt(L[0], L[1], sel);
-  const uint32_t hi = prmt(L[2], L[3], sel);
-  const uint32_t pick = ((x & 0x8888u) >> 1) | 0x3210u;
-  return prmt(lo, hi, pick);
-}
 
 // Eight 4-bit codes (one 32-bit word, code i in bits 4i..4i+3) -> eight LUT
 // bytes: o0 = codes 0-3, o1 = codes 4-7.  prmt reads only the low 16 bits of
@@ -119,17 +113,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
-      "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
-      "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
-      "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
-      : "memory");
-}
 // 32 lanes x 32 bit, 16 consecutive columns -> 16 registers per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -155,7 +138,6 @@ __device__ __forceinline__ void fma_s32x2(float& r0, float& r1, float w0, float 
       : "+f"(r0), "+f"(r1)
       : "r"(x0 + 0x4B400000u), "r"(x1 + 0x4B400000u), "f"(w0), "f"(w1), "f"(12582912.0f));
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Store 32 consecutive outputs of one row (FP32 or BF16), masked to n < N.
 __device__ __forceinline__ void store_row32(void* Y, int out_fp32, int N, int m, int n0, const float (&v)[32]) {
@@ -219,8 +201,14 @@ __device__ __forceinline__ void load_scales_smem(float* slot, const float* src, 
 
 // Epilogue of one 32-column chunk for a finished (non-grouped) accumulator:
 // y = acc * (s_a[m] * s_w[n]) (+ low-rank), stored to Y.
+// With a staging area (two 2 KB buffers per warp, smem address stg) and BF16
+// output, the warp's 32 x 32 block goes to shared memory in the 64-byte
+// swizzled layout of the output tensor map and out with one TMA store; the
+// buffer is rewritten only after the store two chunks back has read it.
 __device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t tacc, uint32_t tlr, bool lr,
-                                                const float* sw, float sa, int row, int nc) {
+                                                const float* sw, float sa, int row, int nc,
+                                                const CUtensorMap* ymap = nullptr, uint32_t stg = 0,
+                                                uint32_t* sc = nullptr, int row0 = 0) {
   uint32_t acc[32];
   tmem_ld32(tacc, acc);
   uint32_t l[32];
@@ -239,7 +227,32 @@ __device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t ta
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += __uint_as_float(l[i]);
   }
-  if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, nc, v);
+  if (stg == 0 || !p.tma_store) {
+    if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, nc, v);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const uint32_t buf = stg + (*sc & 1u) * 2048u;
+  if (*sc >= 2) {
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+  }
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    st_shared_v4(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(ymap, buf, nc, row0);   // rows >= M and columns >= N are clipped by the map
+    bulk_commit_group();
+  }
+  ++*sc;
 }
 
 // ====================================================================== FP8
@@ -252,7 +265,10 @@ __device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t ta
 //   weight-scale slots [2][BN] FP32, barriers, TMEM address, abort flag
 template <int BN, int WBITS>
 struct Fp8Plan {
-  static constexpr int SP = BN == 256 ? 3 : 4, SE = BN == 256 ? 3 : 4;
+  // BN = 256: two expanded stages (the expansion, not the MMA, sets the pace),
+  // a deeper packed ring and 16 KB of output staging for the TMA-store epilogue
+  static constexpr int SP = BN == 256 ? (WBITS == 4 ? 4 : 5) : 4, SE = BN == 256 ? 2 : 4;
+  static constexpr int STG = BN == 256 ? 16384 : 0;   // 4 epilogue warps x 2 x 2 KB
   static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-wide K tile
   static constexpr int PA = BM * 64, PB = BN * WROW, EA = BM * 128, EB = BN * 128;
   static constexpr bool LR = BN == 128;
@@ -264,7 +280,8 @@ struct Fp8Plan {
   static constexpr int OFF_L = OFF_C + (LR ? BM * 64 : 0);
   static constexpr int OFF_SC = OFF_L + (LR ? BN * 64 : 0);
   static constexpr int SCS = BN == 128 ? 12 : 4;               // grouped scale ring depth (BN 128 only)
-  static constexpr int OFF_BAR = OFF_SC + (SCS * BN * 4 > 2 * BN * 4 ? SCS * BN * 4 : 2 * BN * 4);
+  static constexpr int OFF_STG = (OFF_SC + (SCS * BN * 4 > 2 * BN * 4 ? SCS * BN * 4 : 2 * BN * 4) + 1023) & ~1023;
+  static constexpr int OFF_BAR = OFF_STG + STG;
   static constexpr int NBAR = 2 * SP + 2 * SE + 6 + 4 + 2 * SCS;
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(BYTES <= 232448, "shared memory plan exceeds 227 KB");
@@ -451,6 +468,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     const int tid = threadIdx.x - 128;       // 0 .. 32*NEPI-1
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint32_t gc = 0;
+    uint32_t stc = 0;   // TMA-store chunks issued by this warp
+    const uint32_t stg = (!GROUPED && P::STG) ? sbase + P::OFF_STG + (uint32_t)e * 4096u : 0u;
     int tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
@@ -527,7 +546,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
 #pragma unroll 1
         for (int ch = 0; ch < BN / 32; ++ch)
           epi_chunk_final(p, tmem + lane_off + ab * BN + ch * 32, tmem + lane_off + 384 + ch * 32, lr,
-                          sw + ch * 32, sa, row, n0 + ch * 32);
+                          sw + ch * 32, sa, row, n0 + ch * 32, &tm.y, stg, &stc, m0 + q * 32);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -536,6 +555,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         }
       }
     }
+    // the staging buffers must outlive the TMA stores that read them
+    if (P::STG && lane == 0) bulk_wait_group<0>();
   } else if (warp >= EXP0 || (GROUPED && warp >= 2)) {
     // ------------------------------------------------------------ code expansion
     const int t = (GROUPED && warp < 4 ? warp - 2 + (NW - EXP0) : warp - EXP0) * 32 + lane;  // 0 .. NXT-1
@@ -965,6 +986,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   memcpy(gp.w_lut, a.w_lut, 16);
   gp.has_lr = a.c != nullptr;
   gp.Y = a.Y; gp.out_fp32 = a.out_fp32; gp.status = a.status;
+  gp.tma_store = 0;
 
   const bool nvf4 = a.a_fmt == RQ_FMT_NVFP4;
   const bool grouped = a.w_fmt == RQ_FMT_INT4;
@@ -990,6 +1012,12 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     return launch(gemm_nvf4_kernel<128>, Nvf4Plan<128>::BYTES, grid, 256, tm, gp, st);
   }
   const bool w2 = a.w_fmt == RQ_FMT_LM4;
+  if (!grouped && BN == 256 && !a.out_fp32) {
+    // BF16 output through 32 x 32 boxes (the epilogue's TMA stores)
+    ok &= make_map_2d(&tm.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, a.N, a.M, (uint64_t)a.N * 2, 32, 32,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
+    gp.tma_store = 1;
+  }
   ok &= make_map_2d(&tm.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, a.K / 2, a.M, a.K / 2, 64, BM,
                     CU_TENSOR_MAP_SWIZZLE_64B);
   if (w2)
