@@ -266,9 +266,11 @@ __device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t ta
 template <int BN, int WBITS>
 struct Fp8Plan {
   // BN = 256: two expanded stages (the expansion, not the MMA, sets the pace),
-  // a deeper packed ring and 16 KB of output staging for the TMA-store epilogue
-  static constexpr int SP = BN == 256 ? (WBITS == 4 ? 4 : 5) : 4, SE = BN == 256 ? 2 : 4;
-  static constexpr int STG = BN == 256 ? 16384 : 0;   // 4 epilogue warps x 2 x 2 KB
+  // a deeper packed ring and 16 KB of output staging for the TMA-store
+  // epilogue (4 warps x 2 x 2 KB); BN = 128: three expanded stages and 32 KB
+  // of staging (16 grouped epilogue warps x 2 KB, or 4 warps x 2 x 2 KB)
+  static constexpr int SP = BN == 256 ? (WBITS == 4 ? 4 : 5) : 4, SE = BN == 256 ? 2 : 3;
+  static constexpr int STG = BN == 256 ? 16384 : 32768;
   static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-wide K tile
   static constexpr int PA = BM * 64, PB = BN * WROW, EA = BM * 128, EB = BN * 128;
   static constexpr bool LR = BN == 128;
@@ -469,7 +471,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint32_t gc = 0;
     uint32_t stc = 0;   // TMA-store chunks issued by this warp
-    const uint32_t stg = (!GROUPED && P::STG) ? sbase + P::OFF_STG + (uint32_t)e * 4096u : 0u;
+    const uint32_t stg = sbase + P::OFF_STG + (uint32_t)e * (GROUPED ? 2048u : 4096u);
     int tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
@@ -533,7 +535,33 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
 #pragma unroll
           for (int i = 0; i < 32; ++i) run[i] *= sa256;
         }
-        if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, n0 + h * 32, run);
+        if (!p.tma_store) {
+          if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, n0 + h * 32, run);
+        } else {
+          // the warp's 32 x 32 block through shared memory and one TMA store
+          // (single buffer: the previous tile's store has read it long ago)
+          if (stc > 0) {
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            __nv_bfloat162 hb = __floats2bfloat162_rn(run[2 * i], run[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&hb);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                         w[4 * c + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm.y, stg, n0 + h * 32, m0 + q * 32);
+            bulk_commit_group();
+          }
+          ++stc;
+        }
       } else {
         const uint32_t ab = tc & 1;
         float* sw = sc_slots + ab * BN;
@@ -556,7 +584,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
       }
     }
     // the staging buffers must outlive the TMA stores that read them
-    if (P::STG && lane == 0) bulk_wait_group<0>();
+    if (lane == 0) bulk_wait_group<0>();
   } else if (warp >= EXP0 || (GROUPED && warp >= 2)) {
     // ------------------------------------------------------------ code expansion
     const int t = (GROUPED && warp < 4 ? warp - 2 + (NW - EXP0) : warp - EXP0) * 32 + lane;  // 0 .. NXT-1
@@ -1012,7 +1040,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     return launch(gemm_nvf4_kernel<128>, Nvf4Plan<128>::BYTES, grid, 256, tm, gp, st);
   }
   const bool w2 = a.w_fmt == RQ_FMT_LM4;
-  if (!grouped && BN == 256 && !a.out_fp32) {
+  if (!a.out_fp32) {
     // BF16 output through 32 x 32 boxes (the epilogue's TMA stores)
     ok &= make_map_2d(&tm.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, a.N, a.M, (uint64_t)a.N * 2, 32, 32,
                       CU_TENSOR_MAP_SWIZZLE_64B);
