@@ -193,10 +193,10 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int n) {
 // Named barrier among the epilogue warps.
 template <int NT>
 __device__ __forceinline__ void epi_bar_n() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
-__device__ __forceinline__ void epi_bar() { epi_bar_n<128>(); }
 
-__device__ __forceinline__ void load_scales_smem(float* slot, const float* src, int n0, int N, int BNv, int tid) {
-  for (int i = tid; i < BNv; i += 128) slot[i] = n0 + i < N ? __ldg(src + n0 + i) : 0.f;
+__device__ __forceinline__ void load_scales_smem(float* slot, const float* src, int n0, int N, int BNv, int tid,
+                                                 int nthreads = 128) {
+  for (int i = tid; i < BNv; i += nthreads) slot[i] = n0 + i < N ? __ldg(src + n0 + i) : 0.f;
 }
 
 // Epilogue of one 32-column chunk for a finished (non-grouped) accumulator:
@@ -767,8 +767,14 @@ struct Nvf4Plan {
 // from column 256 (BN = 256: 4 slots of 48 columns; BN = 128: 4 slots of 32),
 // one slot per k-tile in flight, so a k-tile's tcgen05.cp never waits for the
 // previous k-tile's MMAs to finish reading their scales.
+// Threads: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warp 2 scale
+// factors -> TMEM, warp 3 idle, warps 4-11 epilogue (two per TMEM lane quadrant,
+// each half of the tile's columns: the BN = 256 accumulator is single-buffered,
+// so the epilogue's length is a pipeline bubble).
+constexpr int NVF4_THREADS = 384;
+
 template <int BN>
-__global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
   using P = Nvf4Plan<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -797,11 +803,11 @@ __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < P::S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 8); }
     mbar_init(lrfull, 1);
     mbar_init(lrsmem_empty, 1);
     mbar_init(lrdone, 1);
-    mbar_init(lracc_empty, 4);
+    mbar_init(lracc_empty, 8);
     for (int i = 0; i < 4; ++i) { mbar_init(&sffull[i], 1); mbar_init(&sfempty[i], 1); }
     *abort_flag = 0;
     fence_mbar_init();
@@ -926,8 +932,9 @@ __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant
       }
     }
   } else if (warp >= 4) {
-    const int q = warp - 4;
-    const int tid = threadIdx.x - 128;
+    const int q = warp & 3;                  // TMEM lane quadrant (warp id % 4)
+    const int half = (warp - 4) >> 2;        // this warp's half of the columns
+    const int tid = threadIdx.x - 128;       // 0 .. 255
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     int tc = 0;
     bool ok = true;
@@ -937,14 +944,14 @@ __global__ void __launch_bounds__(256, 1) gemm_nvf4_kernel(const __grid_constant
       const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
       const uint32_t ab = tc % P::NACC;
       float* sw = sc_slots + (tc & 1) * BN;
-      load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid);
-      epi_bar();
+      load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid, 256);
+      epi_bar_n<256>();
       ok = mbar_wait(&accfull[ab], (tc / P::NACC) & 1, p.status, ST_TIMEOUT_MMA, abort_flag) &&
            (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch)
+      for (int ch = half * (BN / 64); ch < (half + 1) * (BN / 64); ++ch)
         epi_chunk_final(p, tmem + lane_off + ab * BN + ch * 32, tmem + lane_off + 384 + ch * 32, lr, sw + ch * 32,
                         sa, row, n0 + ch * 32);
       tc_fence_before();
@@ -1036,8 +1043,8 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 2, a.N, a.K / 2, 128, BN,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) { *why = "cuTensorMapEncodeTiled failed"; return cudaErrorInvalidValue; }
-    if (BN == 256) return launch(gemm_nvf4_kernel<256>, Nvf4Plan<256>::BYTES, grid, 256, tm, gp, st);
-    return launch(gemm_nvf4_kernel<128>, Nvf4Plan<128>::BYTES, grid, 256, tm, gp, st);
+    if (BN == 256) return launch(gemm_nvf4_kernel<256>, Nvf4Plan<256>::BYTES, grid, NVF4_THREADS, tm, gp, st);
+    return launch(gemm_nvf4_kernel<128>, Nvf4Plan<128>::BYTES, grid, NVF4_THREADS, tm, gp, st);
   }
   const bool w2 = a.w_fmt == RQ_FMT_LM4;
   if (!a.out_fp32) {
