@@ -391,8 +391,7 @@ def run_ours(args, w, rank, world, dist):
 # DRAM bytes per launch of the GEMM (read + write) from a 1-pass ncu capture of
 # the current kernels at the full sizes, keyed by workload (see
 # profiles/dram_traffic_all_workloads.md).
-TRAFFIC = {"c2": 5_790_720 + 37_376, "c3": 21_344_768 + 32_366_848, "c4": 53_147_904 + 3_260_672,
-           "c5": 54_207_232 + 1_119_752_960}
+TRAFFIC = {"c2": 5_847_552, "c3": 55_734_272, "c4": 56_036_096, "c5": 1_174_437_888}
 
 
 def main():
