@@ -28,7 +28,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from rotated_bit_post_b200 import inputs  # noqa: E402
+from rotated_bit_post_b200 import inputs, multirank  # noqa: E402
 
 METRIC = "W4A4 rotated-linear tokens/s & effective TFLOPS (% FP4/FP8 peak) on 1 B200"
 L2_FLUSH_BYTES = 256 << 20
@@ -235,7 +235,7 @@ def run_ours(args, w, rank, world, dist):
                            wb["L"], wb["codes"], wb["scale"], wb["block_scale"], status)
     del Wt
     # this rank's token batch (rank r draws its own tokens)
-    X_np = inputs.activations(w, token_seed=inputs.TOKEN_SEED + rank)
+    X_np = multirank.rank_activations(w, rank)
     X = torch.from_numpy(X_np.view(np.int16)).to(dev)
     ab = rq.act_buffers(w.a_fmt, w.M, w.K, w.rank)
     Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
@@ -282,10 +282,7 @@ def run_ours(args, w, rank, world, dist):
     t_k1 = [e[0].elapsed_time(e[1]) for e in ev]
     t_k2 = [e[1].elapsed_time(e[2]) for e in ev]
     step_ms = sum(a + b for a, b in zip(t_k1, t_k2))
-    if dist is not None:
-        t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = multirank.max_over_ranks(dist, step_ms, dev)
     rc, code = rq.rq_read_status(status)
     if rc != 0:
         raise RuntimeError(f"kernel status {code:#x}")
@@ -336,11 +333,8 @@ def run_ours(args, w, rank, world, dist):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if dist is not None:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": w.M * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": X.numel() * 2,
+        e2e_ms = multirank.max_over_ranks(dist, e2e_ms, dev)
+        e2e = {"value": multirank.aggregate_tokens_per_s(w.M, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": X.numel() * 2,
                "d2h_bytes_per_step": Y.numel() * 2, "ms_per_step": e2e_ms,
                "note": "pinned host X -> device, K1, K2, device Y -> pinned host, per step"}
 
@@ -350,7 +344,7 @@ def run_ours(args, w, rank, world, dist):
     ms_per_step = step_ms / args.steps
     k1_ms = statistics.mean(t_k1)
     k2_ms = statistics.mean(t_k2)
-    tok_s = w.M * world / (ms_per_step * 1e-3)
+    tok_s = multirank.aggregate_tokens_per_s(w.M, world, ms_per_step)
     fl = flops_per_step(w)
     pk = peaks()
     mma_ratio = 4 if w.a_fmt == rq.NVFP4 else 2          # nominal FP4 / FP8 vs BF16 dense ratio
