@@ -41,6 +41,7 @@ namespace {
 
 constexpr int K1_THREADS = 512;
 constexpr int K1_LUT_MAX = 512;
+constexpr int K1_ROW_PAD = 8;   // BF16 elements (16 bytes) after each staged row
 constexpr int K1_WARPS = K1_THREADS / 32;
 
 struct __align__(16) K1Params {
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
   const int K = p.K;
   const int R = p.R;
   const int nblk = K / B;
+  const int KS = PROJ ? K : K + K1_ROW_PAD;   // row stride of the BF16 row buffers
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int lq = lane % L;                 // lane inside its group
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     negc = reinterpret_cast<float*>(smem + off);
     off += (size_t)R * 32 * 4;
   } else {
-    off = (size_t)2 * R * K * 2;
+    off = (size_t)2 * R * (K + K1_ROW_PAD) * 2;
   }
   rot_s = reinterpret_cast<int32_t*>(smem + off);
   off += (size_t)K * 4;
@@ -200,9 +202,9 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
   auto issue_group = [&](int g, int buf) {
     const int r0 = g * R;
     const int nr = min(R, p.rows - r0);
-    uint16_t* dst = PROJ ? land : xs + (size_t)buf * R * K;
+    uint16_t* dst = PROJ ? land : xs + (size_t)buf * R * KS;
     mbar_expect_tx(&full[buf], (uint32_t)nr * row_bytes);
-    for (int i = 0; i < nr; ++i) bulk_g2s(dst + (size_t)i * K, p.x + (size_t)(r0 + i) * K, row_bytes, &full[buf]);
+    for (int i = 0; i < nr; ++i) bulk_g2s(dst + (size_t)i * KS, p.x + (size_t)(r0 + i) * K, row_bytes, &full[buf]);
   };
 
   if (threadIdx.x == 0 && blockIdx.x < p.ngroups) issue_group(blockIdx.x, 0);
@@ -252,7 +254,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
         issue_group(g + gridDim.x, buf ^ 1);
       }
     }
-    const uint16_t* xg = xs + (size_t)buf * R * K;
+    const uint16_t* xg = xs + (size_t)buf * R * KS;
 
     if constexpr (PROJ) {
       // ---------------------------------------------------------- coefficients
@@ -400,6 +402,11 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
       }
     }
 
+    // Items (row, block): without the projection rows vary fastest, so the lane
+    // groups of a warp gather the same columns of consecutive rows, whose
+    // padded buffers (row stride K + 8) put them on different banks.
+    auto item_row = [&](int item) { return PROJ ? item / nblk : item % nr; };
+    auto item_blk = [&](int item) { return PROJ ? item % nblk : item / nr; };
     // ------------------------------------------------------------ phase A
     // gather, transform, block partials; y stays in registers until phase B
     const int nitems = nr * nblk;
@@ -420,7 +427,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     for (int s = 0; s < IPW; ++s) {
       const int item = slot0 + s * SLOTS;
       if (item < nitems) {
-        const int ri = item / nblk, bk = item - ri * nblk;
+        const int ri = item_row(item), bk = item_blk(item);
         const int i0 = bk * B + lq * 32;
         float* v = y[s];
         const int4* rp = reinterpret_cast<const int4*>(rot_s + bk * B + 4 * lq);
@@ -433,7 +440,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
             const int src = rr[q] & 0x7fffffff;
             float xv;
             if constexpr (PROJ) xv = xf[(size_t)ri * K + src];
-            else xv = bf16_bits_to_f32(xg[(size_t)ri * K + src]);
+            else xv = bf16_bits_to_f32(xg[(size_t)ri * KS + src]);
             v[4 * e4 + q] = __uint_as_float(__float_as_uint(xv) ^ ((uint32_t)rr[q] & 0x80000000u));
           }
         }
@@ -504,7 +511,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
 #pragma unroll
       for (int s = 0; s < IPW; ++s) {
         const int item = slot0 + s * SLOTS;
-        if (item < nitems) publish(item / nblk, item % nblk, red[s]);
+        if (item < nitems) publish(item_row(item), item_blk(item), red[s]);
       }
     }
     __syncthreads();
@@ -524,7 +531,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     for (int s = 0; s < IPW; ++s) {
       const int item = slot0 + s * SLOTS;
       if (item < nitems) {
-        const int ri = item / nblk, bk = item - ri * nblk;
+        const int ri = item_row(item), bk = item_blk(item);
         const int row = r0 + ri;
         const int i0 = bk * B + lq * 32;
         float* v = y[s];
@@ -622,7 +629,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
 
 size_t k1_smem_bytes(int R, int K, int nblk, bool proj, int ngrp, int lut_n) {
   size_t off = proj ? (size_t)R * K * 4 + (size_t)32 * ut_pitch(K) * 2 + (size_t)R * 32 * 4
-                    : (size_t)2 * R * K * 2;
+                    : (size_t)2 * R * (K + K1_ROW_PAD) * 2;
   off += (size_t)K * 4;
   off += (size_t)2 * R * nblk * 4;
   off += (size_t)2 * R * ngrp * 4;
