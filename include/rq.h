@@ -27,8 +27,9 @@
  *     stream) and is asynchronous to the host.
  *   - BF16 tensors are passed as their 16-bit patterns (uint16_t).
  *   - Matrices are row-major.  Packed 4-bit codes store element 2j in bits 0-3
- *     and element 2j+1 in bits 4-7 of byte j of the row; packed 2-bit codes store
- *     element 4j+i in bits 2i..2i+1 of byte j.
+ *     and element 2j+1 in bits 4-7 of byte j of the row; packed 2-bit codes go 16
+ *     to a little-endian 32-bit word, nibble i of word w holding element 16w+i in
+ *     bits 0-1 and element 16w+8+i in bits 2-3.
  *   - Argument errors are detected on the host before anything is enqueued and
  *     return RQ_ERR_INVALID_ARG / RQ_ERR_UNSUPPORTED / RQ_ERR_ALIGNMENT with a
  *     message for rq_last_error().  A failed launch returns RQ_ERR_CUDA.

@@ -452,17 +452,22 @@ def unpack_nibbles(p: np.ndarray) -> np.ndarray:
 
 
 def pack_crumbs(q: np.ndarray) -> np.ndarray:
-    """Four 2-bit codes per byte, element 4j+i in bits 2i..2i+1."""
-    q = q.astype(np.uint8) & 3
-    return (q[:, 0::4] | (q[:, 1::4] << 2) | (q[:, 2::4] << 4) | (q[:, 3::4] << 6)).astype(np.uint8)
+    """2-bit codes, 16 per little-endian 32-bit word: element 16w+i (i < 8) in
+    bits 4i..4i+1 of word w, element 16w+8+i in bits 4i+2..4i+3 (nibble i holds
+    elements i and i+8).  Row length a multiple of 16."""
+    q = (q.astype(np.uint8) & 3).reshape(q.shape[0], -1, 16)
+    nib = q[:, :, :8] | (q[:, :, 8:] << 2)                    # nibble i of each word
+    byt = nib[:, :, 0::2] | (nib[:, :, 1::2] << 4)             # byte j = nibbles 2j, 2j+1
+    return byt.reshape(q.shape[0], -1).astype(np.uint8)
 
 
 def unpack_crumbs(p: np.ndarray) -> np.ndarray:
-    p = np.asarray(p, dtype=np.uint8)
-    out = np.empty((p.shape[0], p.shape[1] * 4), dtype=np.uint8)
-    for i in range(4):
-        out[:, i::4] = (p >> (2 * i)) & 3
-    return out
+    p = np.asarray(p, dtype=np.uint8).reshape(p.shape[0], -1, 4)
+    nib = np.empty((p.shape[0], p.shape[1], 8), dtype=np.uint8)
+    nib[:, :, 0::2] = p & 0xF
+    nib[:, :, 1::2] = p >> 4
+    out = np.concatenate([nib & 3, nib >> 2], axis=2)           # elements 0-7, then 8-15
+    return out.reshape(p.shape[0], -1)
 
 
 def int4_from_nibble(n: np.ndarray) -> np.ndarray:

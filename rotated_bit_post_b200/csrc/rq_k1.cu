@@ -587,7 +587,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
             const uint2 cell = lut_s[g];
             const uint32_t c = cell.x + (u >= __uint_as_float(cell.y) ? 1u : 0u);
             if constexpr (FMT == RQ_FMT_LM16) pk[e >> 3] |= c << (4 * (e & 7));
-            else pk[e >> 4] |= c << (2 * (e & 15));
+            else pk[e >> 4] |= c << (4 * (e & 7) + 2 * ((e >> 3) & 1));   // nibble e%8: elements e%8, e%8+8
           }
         } else {  // NVFP4: two 16-element groups per lane
           const float inv_t = mlt;

@@ -91,13 +91,15 @@ __device__ __forceinline__ void lut16x8(uint32_t w, const uint32_t (&L)[4], uint
   o1 = prmt(prmt(L[0], L[1], sel_hi), prmt(L[2], L[3], sel_hi), pick_hi);
 }
 
-// Eight 2-bit codes (bits 0-15 of x) -> eight LUT bytes (lo word: codes 0-3).
-__device__ __forceinline__ void lut4x8(uint32_t x, uint32_t L0, uint32_t& o0, uint32_t& o1) {
-  uint32_t t = (x | (x << 8)) & 0x00FF00FFu;
-  t = (t | (t << 4)) & 0x0F0F0F0Fu;
-  t = (t | (t << 2)) & 0x33333333u;
-  o0 = prmt(L0, 0u, t & 0xFFFFu);
-  o1 = prmt(L0, 0u, t >> 16);
+// Sixteen 2-bit codes (one 32-bit word, nibble i holding codes i and i+8 in
+// bits 0-1 and 2-3) -> sixteen LUT bytes in code order: the two crumbs of every
+// nibble are already prmt selectors.
+__device__ __forceinline__ void lut4x16(uint32_t w, uint32_t L0, uint32_t (&o)[4]) {
+  const uint32_t lo = w & 0x33333333u, hi = (w >> 2) & 0x33333333u;
+  o[0] = prmt(L0, 0u, lo);
+  o[1] = prmt(L0, 0u, lo >> 16);
+  o[2] = prmt(L0, 0u, hi);
+  o[3] = prmt(L0, 0u, hi >> 16);
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -715,8 +717,12 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
             uint32_t o[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              lut4x8(w[j] & 0xFFFFu, LW[0], o[4 * j], o[4 * j + 1]);
-              lut4x8(w[j] >> 16, LW[0], o[4 * j + 2], o[4 * j + 3]);
+              uint32_t q[4];
+              lut4x16(w[j], LW[0], q);
+              o[4 * j] = q[0];
+              o[4 * j + 1] = q[1];
+              o[4 * j + 2] = q[2];
+              o[4 * j + 3] = q[3];
             }
             const uint32_t rowb = eb + r * 128;
 #pragma unroll

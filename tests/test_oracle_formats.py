@@ -84,7 +84,12 @@ def test_pack_layout():
     q = np.array([[1, 2, 3, 4, 15, 0]], dtype=np.uint8)
     assert list(orc.pack_nibbles(q)[0]) == [0x21, 0x43, 0x0F]
     assert np.array_equal(orc.unpack_nibbles(orc.pack_nibbles(q)), q)
-    c = np.array([[1, 2, 3, 0, 3, 3, 3, 3]], dtype=np.uint8)
-    assert list(orc.pack_crumbs(c)[0]) == [0b00111001, 0xFF]
+    # 16 codes per 32-bit word, nibble i = element i (bits 0-1) | element i+8 (bits 2-3)
+    c = np.array([[1, 2, 3, 0, 3, 3, 3, 3, 0, 1, 2, 3, 0, 0, 1, 2]], dtype=np.uint8)
+    # nibbles: 1|0<<2=1, 2|1<<2=6, 3|2<<2=11, 0|3<<2=12, 3|0=3, 3|0=3, 3|1<<2=7, 3|2<<2=11
+    assert list(orc.pack_crumbs(c)[0]) == [0x61, 0xCB, 0x33, 0xB7]
     assert np.array_equal(orc.unpack_crumbs(orc.pack_crumbs(c)), c)
+    rng = np.random.default_rng(5)
+    c2 = rng.integers(0, 4, size=(3, 64)).astype(np.uint8)
+    assert np.array_equal(orc.unpack_crumbs(orc.pack_crumbs(c2)), c2)
     assert list(orc.int4_from_nibble(np.array([0, 7, 8, 9, 15], np.uint8))) == [0, 7, -8, -7, -1]
