@@ -265,16 +265,20 @@ __device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t ta
 //   e4m3 B    [SE][BN x 128 B]
 //   c / L     [128 x 64 B] / [BN x 64 B] (64B swizzle, BN == 128 only)
 //   weight-scale slots [2][BN] FP32, barriers, TMEM address, abort flag
-template <int BN, int WBITS>
+template <int BN, int WBITS, bool PAIR = false>
 struct Fp8Plan {
   // BN = 256: two expanded stages (the expansion, not the MMA, sets the pace),
   // a deeper packed ring and 16 KB of output staging for the TMA-store
   // epilogue (4 warps x 2 x 2 KB); BN = 128: three expanded stages and 32 KB
-  // of staging (16 grouped epilogue warps x 2 KB, or 4 warps x 2 x 2 KB)
-  static constexpr int SP = BN == 256 ? (WBITS == 4 ? 4 : 5) : 4, SE = BN == 256 ? 2 : 3;
+  // of staging (16 grouped epilogue warps x 2 KB, or 4 warps x 2 x 2 KB).
+  // PAIR (a CTA pair sharing 256 x 256 tiles): each CTA holds half of the
+  // tile's weight rows, so four expanded stages fit.
+  static constexpr int BR = PAIR ? BN / 2 : BN;       // weight rows held by this CTA
+  static constexpr int SP = PAIR ? 4 : BN == 256 ? (WBITS == 4 ? 4 : 5) : 4;
+  static constexpr int SE = PAIR ? 4 : BN == 256 ? 2 : 3;
   static constexpr int STG = BN == 256 ? 16384 : 32768;
   static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-wide K tile
-  static constexpr int PA = BM * 64, PB = BN * WROW, EA = BM * 128, EB = BN * 128;
+  static constexpr int PA = BM * 64, PB = BR * WROW, EA = BM * 128, EB = BR * 128;
   static constexpr bool LR = BN == 128;
   static constexpr int OFF_PA = 0;
   static constexpr int OFF_PB = OFF_PA + SP * PA;
@@ -306,9 +310,10 @@ struct Fp8Plan {
 template <int BN, bool GROUPED>
 constexpr int fp8_threads() { return GROUPED ? 704 : BN == 256 ? 768 : 512; }
 
-template <int BN, int WBITS, bool GROUPED>
+template <int BN, int WBITS, bool GROUPED, bool PAIR = false>
 __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
-  using P = Fp8Plan<BN, WBITS>;
+  static_assert(!PAIR || (BN == 256 && !GROUPED), "CTA pairs run the 256-wide codebook tiles only");
+  using P = Fp8Plan<BN, WBITS, PAIR>;
   constexpr int NW = fp8_threads<BN, GROUPED>() / 32;
   constexpr int NEPI = GROUPED ? 16 : 4;         // epilogue warps
   constexpr int EXP0 = 4 + NEPI;                 // first expansion warp
@@ -339,13 +344,22 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
   const int nk = p.K / 128;                // 128-wide K tiles == INT4 groups
   constexpr bool grouped = GROUPED;
   const bool lr = P::LR && p.has_lr;
-  const int nN = (p.N + BN - 1) / BN, nM = (p.M + BM - 1) / BM;
+  // PAIR: the two CTAs of a cluster share 256 x BN tiles; CTA `crank` takes
+  // rows crank*128 .. +127 of the tile and weight rows crank*BN/2 .. +BN/2-1,
+  // and the even CTA issues the pair's MMAs.
+  const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
+  constexpr int TM = PAIR ? 2 * BM : BM;
+  const int nN = (p.N + BN - 1) / BN, nM = (p.M + TM - 1) / TM;
   const int ntiles = nM * nN;
+  const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < P::SP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], NXW); }
-    for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], NXW); mbar_init(&eempty[i], 1); }
-    for (int i = 0; i < 3; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], NEPI); }
+    // PAIR: efull / accempty of the even CTA count both CTAs' warps; eempty and
+    // accfull take one multicast commit arrival in each CTA
+    for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], PAIR ? 2 * NXW : NXW); mbar_init(&eempty[i], 1); }
+    for (int i = 0; i < 3; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], PAIR ? 2 * NEPI : NEPI); }
     mbar_init(lrfull, 1);
     mbar_init(lrsmem_empty, 1);
     mbar_init(lrdone, 1);
@@ -357,11 +371,19 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     prefetch_tmap(&tm.b);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc2(tmem_slot, 512);
+      tmem_relinquish2();
+    } else {
+      tmem_alloc(tmem_slot, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();   // both CTAs' barriers exist before either arrives on the other's
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -371,8 +393,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
       uint32_t kc = 0;
       int tc = 0;
       uint32_t sgc = 0;                    // group-scale ring counter (GROUPED)
-      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
-        const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+      for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep, ++tc) {
+        const int m0 = (tile / nN) * TM + (int)crank * BM, n0 = (tile % nN) * BN;
         for (int kt = 0; kt < nk; ++kt, ++kc) {
           if constexpr (GROUPED) {
             // this group's weight scales s_w[kt, n0 .. n0+127] (one contiguous row slice)
@@ -387,7 +409,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           if (kc >= P::SP && !mbar_wait(&pempty[s], ((kc / P::SP) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
           mbar_expect_tx(&pfull[s], P::PA + P::PB);
           tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * 64, m0, &pfull[s]);
-          tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0, &pfull[s]);
+          tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0 + (int)crank * P::BR, &pfull[s]);
         }
         // the tile's low-rank operands go after its K tiles, so waiting for the
         // previous tile's low-rank MMA never stalls the K-tile prefetch
@@ -401,8 +423,10 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = GROUPED ? idesc_i8(BN) : idesc_f8(BN);
+    if (lane == 0 && crank == 0) {
+      // (PAIR: M = 256, the instruction descriptor's M field is M / 16)
+      const uint32_t idesc =
+          GROUPED ? idesc_i8(BN) : PAIR ? (idesc_f8(BN) & ~(0x1Fu << 24)) | (16u << 24) : idesc_f8(BN);
       uint32_t kc = 0, gc = 0;
       int tc = 0;
       bool ok = true;
@@ -422,7 +446,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         tc_commit(lrsmem_empty);
         return true;
       };
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+      for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
         const uint32_t ab = tc & 1;
         if (!grouped && tc >= 2) {
           ok = mbar_wait(&accempty[ab], ((tc >> 1) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag);
@@ -450,18 +474,27 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
             if constexpr (GROUPED)
               umma_i8(tmem + buf * 128, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
                       idesc, (fresh && kk == 0) ? 0u : 1u);
+            else if constexpr (PAIR)
+              umma_f8_2(tmem + buf * BN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
+                        idesc, (fresh && kk == 0) ? 0u : 1u);
             else
               umma_f8(tmem + buf * BN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
                       idesc, (fresh && kk == 0) ? 0u : 1u);
           }
-          tc_commit(&eempty[s]);
+          if constexpr (PAIR)
+            tc_commit2_mc(&eempty[s], 0x3);   // the stage is free in both CTAs
+          else
+            tc_commit(&eempty[s]);
           if (grouped) {
             tc_commit(&accfull[buf]);
             ++gc;
           }
         }
         if (!ok) break;
-        if (!grouped) tc_commit(&accfull[ab]);
+        if constexpr (PAIR)
+          tc_commit2_mc(&accfull[ab], 0x3);
+        else if (!grouped)
+          tc_commit(&accfull[ab]);
         if (lr && !(ok = lowrank(tc))) break;
       }
     }
@@ -476,8 +509,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     const uint32_t stg = sbase + P::OFF_STG + (uint32_t)e * (GROUPED ? 2048u : 4096u);
     int tc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
-      const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
+    for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
+      const int m0 = (tile / nN) * TM + (int)crank * BM, n0 = (tile % nN) * BN;
       const int row = m0 + q * 32 + lane;
       const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
       if constexpr (GROUPED) {
@@ -580,7 +613,10 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&accempty[ab]);
+          if constexpr (PAIR)
+            mbar_arrive_cluster(&accempty[ab], 0);
+          else
+            mbar_arrive(&accempty[ab]);
           if (lr) mbar_arrive(lracc_empty);
         }
       }
@@ -598,7 +634,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     }
     uint32_t kc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
       for (int kt = 0; kt < nk; ++kt, ++kc) {
         const int sp = kc % P::SP, se = kc % P::SE;
         ok = mbar_wait(&pfull[sp], (kc / P::SP) & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
@@ -675,18 +711,18 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
         }
         if constexpr (WBITS == 4) {
-          constexpr int NBI = (BN * 4 + NXT - 1) / NXT;
+          constexpr int NBI = (P::BR * 4 + NXT - 1) / NXT;
           uint4 vb[NBI];
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
             const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-            if (idx < BN * 4) vb[it] = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+            if (idx < P::BR * 4) vb[it] = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
           }
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
-            if (idx >= BN * 4) break;
+            if (idx >= P::BR * 4) break;
             const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
             const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -699,18 +735,18 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           }
         } else {
           // 2-bit weights: 32 packed bytes per row = 2 segments of 64 codes
-          constexpr int NBI = (BN * 2 + NXT - 1) / NXT;
+          constexpr int NBI = (P::BR * 2 + NXT - 1) / NXT;
           uint4 vb[NBI];
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
             const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
-            if (idx < BN * 2) vb[it] = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
+            if (idx < P::BR * 2) vb[it] = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
           }
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
             const int idx = it * NXT + t;
-            if (idx >= BN * 2) break;
+            if (idx >= P::BR * 2) break;
             const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
             const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -733,18 +769,35 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         fence_proxy_async_smem();  // make the generic-proxy writes visible to the tensor core
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&efull[se]);
+          if constexpr (PAIR)
+            mbar_arrive_cluster(&efull[se], 0);   // the even CTA's MMA waits for both halves
+          else
+            mbar_arrive(&efull[se]);
           mbar_arrive(&pempty[sp]);
         }
       }
     }
+    if constexpr (PAIR) {
+      // the even CTA's last commits land in this CTA's barriers: wait for them
+      // before this CTA may leave
+      for (uint32_t c = kc > (uint32_t)P::SE ? kc - P::SE : 0; ok && c < kc; ++c)
+        ok = mbar_wait(&eempty[c % P::SE], (c / P::SE) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag);
+    }
   }
 
   tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+  if constexpr (PAIR) {
+    cluster_sync();   // neither CTA leaves while the other may still touch its barriers
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc2(tmem, 512);
+    }
+  } else {
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
   }
 }
 
@@ -1013,6 +1066,41 @@ cudaError_t launch(Kern k, int smem, dim3 grid, int threads, const TMaps& tm, co
   return cudaGetLastError();
 }
 
+// CTA-pair kernels: clusters of two, as many pairs as can be resident at once
+// (at most `pairs`).
+template <class Kern>
+cudaError_t launch_pair(Kern k, int smem, int pairs, int threads, const TMaps& tm, const GemmParams& gp,
+                        cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static const void* cached_k[8] = {};
+  static int cached_n[8] = {};
+  int resident = 0;
+  for (int i = 0; i < 8; ++i)
+    if (cached_k[i] == (const void*)k) resident = cached_n[i];
+  if (resident == 0) {
+    e = cudaOccupancyMaxActiveClusters(&resident, k, &cfg);
+    if (e != cudaSuccess) return e;
+    if (resident < 1) return cudaErrorInvalidConfiguration;
+    for (int i = 0; i < 8; ++i)
+      if (!cached_k[i]) { cached_k[i] = (const void*)k; cached_n[i] = resident; break; }
+  }
+  cfg.gridDim = dim3(2 * (pairs < resident ? pairs : resident));
+  return cudaLaunchKernelEx(&cfg, k, tm, gp);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) {
@@ -1061,17 +1149,26 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   }
   ok &= make_map_2d(&tm.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, a.K / 2, a.M, a.K / 2, 64, BM,
                     CU_TENSOR_MAP_SWIZZLE_64B);
+  // 256-wide codebook tiles run on CTA pairs (256 x 256 per pair, each CTA
+  // loading and expanding half of the weight rows)
+  const bool pair = !grouped && BN == 256;
+  const uint32_t brows = pair ? BN / 2 : BN;
   if (w2)
-    ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 4, a.N, a.K / 4, 32, BN,
+    ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 4, a.N, a.K / 4, 32, brows,
                       CU_TENSOR_MAP_SWIZZLE_32B);
   else
-    ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 2, a.N, a.K / 2, 64, BN,
+    ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 2, a.N, a.K / 2, 64, brows,
                       CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) { *why = "cuTensorMapEncodeTiled failed"; return cudaErrorInvalidValue; }
   if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<128, true>(), tm, gp, st);
-  if (BN == 256) {
-    if (w2) return launch(gemm_fp8_kernel<256, 2, false>, Fp8Plan<256, 2>::BYTES, grid, fp8_threads<256, false>(), tm, gp, st);
-    return launch(gemm_fp8_kernel<256, 4, false>, Fp8Plan<256, 4>::BYTES, grid, fp8_threads<256, false>(), tm, gp, st);
+  if (pair) {
+    const int ptiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+    const int pairs = ptiles < sms / 2 ? ptiles : sms / 2;
+    if (w2)
+      return launch_pair(gemm_fp8_kernel<256, 2, false, true>, Fp8Plan<256, 2, true>::BYTES, pairs,
+                         fp8_threads<256, false>(), tm, gp, st);
+    return launch_pair(gemm_fp8_kernel<256, 4, false, true>, Fp8Plan<256, 4, true>::BYTES, pairs,
+                       fp8_threads<256, false>(), tm, gp, st);
   }
   if (w2) return launch(gemm_fp8_kernel<128, 2, false>, Fp8Plan<128, 2>::BYTES, grid, fp8_threads<128, false>(), tm, gp, st);
   return launch(gemm_fp8_kernel<128, 4, false>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<128, false>(), tm, gp, st);
