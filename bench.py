@@ -15,6 +15,7 @@ the host cores on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -44,6 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bf16-linear", action="store_true", help="skip the cuBLAS BF16 linear on the same shapes")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="token rows per rank (default: the workload's own); smaller cases for profiler captures")
     return ap.parse_args()
 
 
@@ -248,10 +251,10 @@ def run_ours(args, w, rank, world, dist):
         rq.rq_rotate_quantize_act(w.a_fmt, x, w.block, rot_t, a_bnd, U_t, ab["c"], ab["codes"], ab["scale"],
                                   ab["block_scale"], status, stream)
 
-    def k2():
+    def k2(y=None):
         rq.rq_w4a4_linear(w.a_fmt, w.w_fmt, w.M, w.N, w.K, ab["codes"], ab["scale"], ab["block_scale"],
-                          wb["codes"], wb["scale"], wb["block_scale"], a_lut, w_lut, ab["c"], wb["L"], Y, 0,
-                          status, stream)
+                          wb["codes"], wb["scale"], wb["block_scale"], a_lut, w_lut, ab["c"], wb["L"],
+                          Y if y is None else y, 0, status, stream)
 
     def barrier():
         if dist is not None:
@@ -310,33 +313,64 @@ def run_ours(args, w, rank, world, dist):
         del Wb, Yb
 
     # ---------------- end to end through the public API with host buffers
+    # Every step copies its token batch from pinned host memory to the device,
+    # runs K1 and K2, and copies its BF16 output back to pinned host memory.
+    # The copies run on their own streams, double-buffered, so that step i+1's
+    # upload and step i-1's download overlap step i's kernels (PCIe is full
+    # duplex); the timed region spans the first upload to the last download.
     e2e = None
     if not args.no_e2e:
         X_host = torch.from_numpy(X_np.view(np.int16)).pin_memory()
         Y_host = torch.empty((w.M, w.N), dtype=torch.bfloat16).pin_memory()
-        Xd = torch.empty_like(X)
+        Xd = [torch.empty_like(X), torch.empty_like(X)]
+        Yd = [Y, torch.empty_like(Y)]
+        s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         n_e2e = max(5, min(50, args.steps))
-        for _ in range(3):
-            Xd.copy_(X_host, non_blocking=True)
-            k1(Xd)
-            k2()
-            Y_host.copy_(Y, non_blocking=True)
+
+        def run_steps(n, e_first=None, e_last=None):
+            up_done = [torch.cuda.Event() for _ in range(n)]
+            x_free = [torch.cuda.Event() for _ in range(n)]
+            comp_done = [torch.cuda.Event() for _ in range(n)]
+            down_done = [torch.cuda.Event() for _ in range(n)]
+            if e_first is not None:
+                e_first.record(s_up)
+            for i in range(n):
+                b = i & 1
+                with torch.cuda.stream(s_up):
+                    if i >= 2:
+                        s_up.wait_event(x_free[i - 2])
+                    Xd[b].copy_(X_host, non_blocking=True)
+                    up_done[i].record(s_up)
+                stream.wait_event(up_done[i])
+                if i >= 2:
+                    stream.wait_event(down_done[i - 2])
+                k1(Xd[b])
+                x_free[i].record(stream)
+                k2(Yd[b])
+                comp_done[i].record(stream)
+                with torch.cuda.stream(s_down):
+                    s_down.wait_event(comp_done[i])
+                    Y_host.copy_(Yd[b], non_blocking=True)
+                    down_done[i].record(s_down)
+            if e_last is not None:
+                e_last.record(s_down)
+
+        run_steps(3)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            Xd.copy_(X_host, non_blocking=True)
-            k1(Xd)
-            k2()
-            Y_host.copy_(Y, non_blocking=True)
-        e1.record(stream)
+        run_steps(n_e2e, e0, e1)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / n_e2e
         e2e_ms = multirank.max_over_ranks(dist, e2e_ms, dev)
+        rc, code = rq.rq_read_status(status)
+        if rc != 0:
+            raise RuntimeError(f"kernel status {code:#x}")
         e2e = {"value": multirank.aggregate_tokens_per_s(w.M, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": X.numel() * 2,
                "d2h_bytes_per_step": Y.numel() * 2, "ms_per_step": e2e_ms,
-               "note": "pinned host X -> device, K1, K2, device Y -> pinned host, per step"}
+               "note": "per step: pinned host X -> device, K1, K2, device Y -> pinned host; uploads and "
+                       "downloads on their own streams overlap the neighbouring steps' kernels"}
+        del Xd, Yd
 
     if rank != 0:
         return
@@ -358,7 +392,7 @@ def run_ours(args, w, rank, world, dist):
                 "peak": tensor_peak, "unit": "TFLOP/s", "frac": k2_tflops / tensor_peak,
                 "peak_source": f"{pk['source']} bf16 burst {pk['bf16_tflops']} x nominal ratio {mma_ratio} "
                                f"({'fp4' if mma_ratio == 4 else 'fp8'}/bf16)",
-                "algorithmic_per_launch": f"{fl:.4g} FLOP (2MNK + 2MNr)", "traffic": TRAFFIC.get(w.name)}
+                "algorithmic_per_launch": f"{fl:.4g} FLOP (2MNK + 2MNr)", "traffic": None if args.tokens else TRAFFIC.get(w.name)}
     else:
         roof = {"kernel": "rq_rotate_quantize_act", "bound": "hbm", "achieved": k1_gbs, "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": k1_gbs / pk["hbm_gbs"], "peak_source": pk["source"] + " copy",
@@ -385,12 +419,14 @@ def run_ours(args, w, rank, world, dist):
 # DRAM bytes per launch of the GEMM (read + write) from a 1-pass ncu capture of
 # the current kernels at the full sizes, keyed by workload (see
 # profiles/dram_traffic_all_workloads.md).
-TRAFFIC = {"c2": 5_847_552, "c3": 55_734_272, "c4": 56_036_096, "c5": 1_174_437_888}
+TRAFFIC = {"c2": 5_847_552, "c3": 55_207_424, "c4": 56_036_096, "c5": 1_174_680_064}
 
 
 def main():
     args = parse()
     w = inputs.WORKLOADS[args.config]
+    if args.tokens:
+        w = dataclasses.replace(w, M=args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
