@@ -112,6 +112,19 @@ __device__ __forceinline__ void fma2(float& v0, float& v1, uint64_t s2, float o0
       "fma.rn.f32x2 v, %2, v, o;\n\tmov.b64 {%0, %1}, v;\n\t}"
       : "+f"(v0), "+f"(v1) : "l"(s2), "f"(o0), "f"(o1));
 }
+// acc (two FP32 in one 64-bit register) = (c, c) * u2 + acc: one IEEE FMA per
+// element, c broadcast, u2 two packed FP32 values
+__device__ __forceinline__ void fma2_bcast(uint64_t& acc, float c, uint64_t u2) {
+  asm("{\n\t.reg .b64 cc;\n\tmov.b64 cc, {%1, %1};\n\tfma.rn.f32x2 %0, cc, %2, %0;\n\t}"
+      : "+l"(acc)
+      : "f"(c), "l"(u2));
+}
+// the two BF16 halves of a word, widened to FP32 and packed (low half first)
+__device__ __forceinline__ uint64_t widen2(uint32_t w) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
 // v = v * s on two elements, s a packed pair
 __device__ __forceinline__ void mul2(float& v0, float& v1, uint64_t s2) {
   asm("{\n\t.reg .b64 v;\n\tmov.b64 v, {%0, %1};\n\tmul.rn.f32x2 v, v, %2;\n\tmov.b64 {%0, %1}, v;\n\t}"
@@ -348,14 +361,12 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
           // block's U^T words and -c vectors are loaded one block ahead.
           const int n = rb - ra;
           const float4* c4[4];
-          float va[4], vb[4];
+          uint64_t vab[4];   // (x[k], x[k+1]) of each row, packed: both chains in one FMA
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const int rr = ra + (r < n ? r : 0);
             c4[r] = reinterpret_cast<const float4*>(negc + rr * 32);
-            const float2 x2 = *reinterpret_cast<const float2*>(xf + (size_t)rr * K + k);
-            va[r] = x2.x;
-            vb[r] = x2.y;
+            vab[r] = *reinterpret_cast<const uint64_t*>(xf + (size_t)rr * K + k);
           }
           const uint16_t* uk = ut + k;
           uint32_t wn[4];
@@ -366,13 +377,10 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
           for (int r = 0; r < 4; ++r) cn[r] = c4[r][0];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            float ua[4], ub[4];
+            uint64_t u2[4];   // (U[k][j], U[k+1][j]) for the four j of this block
             float4 cc[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              ua[i] = __uint_as_float(wn[i] << 16);
-              ub[i] = __uint_as_float(wn[i] & 0xFFFF0000u);
-            }
+            for (int i = 0; i < 4; ++i) u2[i] = widen2(wn[i]);
 #pragma unroll
             for (int r = 0; r < 4; ++r) cc[r] = cn[r];
             if (q < 7) {
@@ -382,21 +390,17 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
               for (int r = 0; r < 4; ++r) cn[r] = c4[r][q + 1];
             }
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              va[r] = __fmaf_rn(cc[r].x, ua[0], va[r]);     // exact products
-              vb[r] = __fmaf_rn(cc[r].x, ub[0], vb[r]);
-              va[r] = __fmaf_rn(cc[r].y, ua[1], va[r]);
-              vb[r] = __fmaf_rn(cc[r].y, ub[1], vb[r]);
-              va[r] = __fmaf_rn(cc[r].z, ua[2], va[r]);
-              vb[r] = __fmaf_rn(cc[r].z, ub[2], vb[r]);
-              va[r] = __fmaf_rn(cc[r].w, ua[3], va[r]);
-              vb[r] = __fmaf_rn(cc[r].w, ub[3], vb[r]);
+            for (int r = 0; r < 4; ++r) {   // exact products; j in order per chain
+              fma2_bcast(vab[r], cc[r].x, u2[0]);
+              fma2_bcast(vab[r], cc[r].y, u2[1]);
+              fma2_bcast(vab[r], cc[r].z, u2[2]);
+              fma2_bcast(vab[r], cc[r].w, u2[3]);
             }
           }
           // rows past the set's end computed a copy of its first row: not stored
 #pragma unroll
           for (int r = 0; r < 4; ++r)
-            if (r < n) *reinterpret_cast<float2*>(xf + (size_t)(ra + r) * K + k) = make_float2(va[r], vb[r]);
+            if (r < n) *reinterpret_cast<uint64_t*>(xf + (size_t)(ra + r) * K + k) = vab[r];
         }
         __syncthreads();
       }
@@ -428,7 +432,6 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
       const int item = slot0 + s * SLOTS;
       if (item < nitems) {
         const int ri = item_row(item), bk = item_blk(item);
-        const int i0 = bk * B + lq * 32;
         float* v = y[s];
         const int4* rp = reinterpret_cast<const int4*>(rot_s + bk * B + 4 * lq);
 #pragma unroll
