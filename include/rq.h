@@ -33,6 +33,8 @@
  *   - Argument errors are detected on the host before anything is enqueued and
  *     return RQ_ERR_INVALID_ARG / RQ_ERR_UNSUPPORTED / RQ_ERR_ALIGNMENT with a
  *     message for rq_last_error().  A failed launch returns RQ_ERR_CUDA.
+ *   - An empty batch (zero token rows, zero weight rows, M = 0) passes the same
+ *     argument checks and returns RQ_OK without enqueuing anything.
  *   - `status` (device int32, caller-initialised to 0) receives a non-zero code
  *     if a kernel gave up a bounded wait; read it back with rq_read_status().
  *     Kernels never wait without bound.

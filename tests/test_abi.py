@@ -92,3 +92,22 @@ def test_argument_errors_are_host_side(L):
     assert code == 1
     code = L.rq_make_codebook(1152, 8, None, None, None, None)
     assert code == 2
+
+
+def test_empty_batch_is_a_noop(L):
+    # zero token rows (or zero weight rows) pass every argument check and return
+    # RQ_OK without touching the (here fake, 16-byte aligned) device pointers
+    p = ctypes.c_void_p(0x1000)
+    code = L.rq_rotate_quantize_act(rq.INT4, p, 0, 1152, 128, p, None, None, 0, None, p, p, None, None, None)
+    assert code == 0, rq.rq_last_error()
+    code = L.rq_rotate_quantize_act(rq.NVFP4, p, 0, 1024, 256, p, None, None, 0, None, p, p, p, None, None)
+    assert code == 0, rq.rq_last_error()
+    code = L.rq_quantize_weights(rq.LM4, p, 0, 1536, 128, p, p, None, 0, None, p, p, None, None, None)
+    assert code == 0, rq.rq_last_error()
+    code = L.rq_w4a4_linear(rq.LM16, rq.LM4, 0, 256, 1536, p, p, None, p, p, None, p, p, None, None, 0, p, 0,
+                            None, None)
+    assert code == 0, rq.rq_last_error()
+    # a negative count is still an error
+    code = L.rq_w4a4_linear(rq.LM16, rq.LM4, -1, 256, 1536, p, p, None, p, p, None, p, p, None, None, 0, p, 0,
+                            None, None)
+    assert code == 1
