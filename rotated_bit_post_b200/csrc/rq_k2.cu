@@ -31,6 +31,7 @@
 //    added after the per-token scale.
 // Every mbarrier wait is bounded (see rq_ptx.cuh); a timeout is reported through
 // the caller's status word and all warps leave together.
+#include <mutex>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -1085,17 +1086,28 @@ cudaError_t launch_pair(Kern k, int smem, int pairs, int threads, const TMaps& t
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // resident-pair counts per kernel, computed once (guarded: host threads may
+  // launch concurrently)
+  static std::mutex mu;
   static const void* cached_k[8] = {};
   static int cached_n[8] = {};
   int resident = 0;
-  for (int i = 0; i < 8; ++i)
-    if (cached_k[i] == (const void*)k) resident = cached_n[i];
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < 8; ++i)
+      if (cached_k[i] == (const void*)k) resident = cached_n[i];
+  }
   if (resident == 0) {
     e = cudaOccupancyMaxActiveClusters(&resident, k, &cfg);
     if (e != cudaSuccess) return e;
     if (resident < 1) return cudaErrorInvalidConfiguration;
+    std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < 8; ++i)
-      if (!cached_k[i]) { cached_k[i] = (const void*)k; cached_n[i] = resident; break; }
+      if (!cached_k[i] || cached_k[i] == (const void*)k) {
+        cached_k[i] = (const void*)k;
+        cached_n[i] = resident;
+        break;
+      }
   }
   cfg.gridDim = dim3(2 * (pairs < resident ? pairs : resident));
   return cudaLaunchKernelEx(&cfg, k, tm, gp);
