@@ -14,6 +14,9 @@
 //    code into its exactly representable E4M3 byte through a 16-entry byte LUT
 //    (prmt) and write the 128-byte-swizzled K-major operand tiles that
 //    tcgen05.mma.kind::f8f6f4 reads; one thread issues the MMAs into TMEM.
+//    The 256-wide tiles run on CTA pairs (cta_group::2, M = 256): each CTA of a
+//    cluster of two loads and expands its own 128 token rows and half of the
+//    tile's weight rows, and the even CTA issues the pair's MMAs.
 //  * INT4 path: a two's-complement nibble v placed in the high half of a byte
 //    is the int8 value 16 v, so expansion is two masks and a shift per eight
 //    codes (even and odd codes land in separate words; A and B use the same
