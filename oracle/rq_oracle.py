@@ -23,7 +23,7 @@ What it computes, in plain numpy, step by step as the pages state it:
   quantized (DiRotQ abstract);
 * the FP64 reference GEMM over the dequantized values.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 FP32 arithmetic with round-to-nearest-even and no fused multiply-add except
 where a product is exact; butterfly stages in ascending stride; a perfect
 pairwise sum of squares inside each block and a sequential sum over blocks;
