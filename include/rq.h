@@ -29,7 +29,9 @@
  *   - Matrices are row-major.  Packed 4-bit codes store element 2j in bits 0-3
  *     and element 2j+1 in bits 4-7 of byte j of the row; packed 2-bit codes go 16
  *     to a little-endian 32-bit word, nibble i of word w holding element 16w+i in
- *     bits 0-1 and element 16w+8+i in bits 2-3.
+ *     bits 0-1 and element 16w+8+i in bits 2-3.  A 16-level codebook code c
+ *     (the count of boundaries at or below the value) is stored in its nibble
+ *     sign-magnitude: c - 8 for c >= 8, (7 - c) | 8 below the centre.
  *   - Argument errors are detected on the host before anything is enqueued and
  *     return RQ_ERR_INVALID_ARG / RQ_ERR_UNSUPPORTED / RQ_ERR_ALIGNMENT with a
  *     message for rq_last_error().  A failed launch returns RQ_ERR_CUDA.
@@ -58,7 +60,7 @@ typedef int32_t rq_status;
 
 /* Quantization formats. */
 #define RQ_INT4 1  /* symmetric INT4 in -7..7, two's-complement nibbles          */
-#define RQ_LM16 2  /* 16-level Lloyd-Max codebook index, nibbles                  */
+#define RQ_LM16 2  /* 16-level Lloyd-Max codebook index, sign-magnitude nibbles   */
 #define RQ_NVFP4 3 /* E2M1 nibbles + UE4M3 block scale per 16 + FP32 row scale    */
 #define RQ_LM4 4   /* 4-level Lloyd-Max codebook index, 2-bit (weights only)       */
 
@@ -177,6 +179,9 @@ rq_status rq_quantize_weights(int32_t fmt, const uint16_t* W, int32_t N, int32_t
  *   a_codes/w_codes, a_scale/w_scale, a_bscale/w_bscale: as produced above.
  *   a_lut/w_lut  [host, 16 / 4 bytes] E4M3 value of each codebook index
  *          (rq_make_codebook's centroids_e4m3) for LM formats; NULL otherwise.
+ *          Read during the argument checks.  A 16-entry table must be
+ *          symmetric (entry 7-m = entry 8+m with the sign bit set), which the
+ *          symmetric Lloyd-Max codebook is; otherwise RQ_ERR_UNSUPPORTED.
  *   c, L, r  [device] low-rank branch (r == 32) or NULL / 0.
  *   Y      [device, M x N] FP32 (out_fp32 = 1) or BF16 (out_fp32 = 0).
  *   Shapes: M >= 1, N % 32 == 0, K % 128 == 0 (K % 256 == 0 for NVFP4).

@@ -443,6 +443,24 @@ def pack_nibbles(q: np.ndarray) -> np.ndarray:
     return (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
 
 
+def sign_magnitude16(q: np.ndarray) -> np.ndarray:
+    """The stored form of a 16-level codebook code c (0..15, the count of
+    boundaries at or below u).  The codebook of the symmetric marginal is
+    symmetric (centroid 15-c = -centroid c), so c is stored as its distance from
+    the centre, m = c - 8 for c >= 8 and 7 - c below (bits 0-2), with bit 3 set
+    for the lower half: centroid(c) = (bit 3 ? -1 : +1) * centroid(8 + m).  The
+    pages fix no bit layout for packed codes; this one lets a consumer read one
+    8-entry magnitude table."""
+    c = np.asarray(q, dtype=np.int16)
+    return np.where(c >= 8, c - 8, (7 - c) | 8).astype(np.uint8)
+
+
+def code_from_sign_magnitude16(d: np.ndarray) -> np.ndarray:
+    """Inverse of sign_magnitude16."""
+    d = np.asarray(d, dtype=np.int16)
+    return np.where(d >= 8, 7 - (d & 7), 8 + d).astype(np.uint8)
+
+
 def unpack_nibbles(p: np.ndarray) -> np.ndarray:
     p = np.asarray(p, dtype=np.uint8)
     out = np.empty((p.shape[0], p.shape[1] * 2), dtype=np.uint8)
@@ -508,7 +526,7 @@ def rotate_quantize(x_bf16_f32: np.ndarray, fmt: int, block: int, sign, perm,
     elif fmt in (LM16, LM4):
         q, s = quant_codebook(y, block, boundaries_f32)
         out["q"], out["scale"] = q, s
-        out["codes"] = pack_crumbs(q) if fmt == LM4 else pack_nibbles(q)
+        out["codes"] = pack_crumbs(q) if fmt == LM4 else pack_nibbles(sign_magnitude16(q))
     elif fmt == NVFP4:
         q, sb, s = quant_nvfp4(y)
         out["q"], out["codes"], out["block_scale"], out["scale"] = q, pack_nibbles(q), sb, s

@@ -164,6 +164,17 @@ rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int
   if (a_fmt == RQ_NVFP4 && (!a_bscale || !w_bscale)) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs block scales");
   if (a_fmt == RQ_LM16 && (!a_lut || !w_lut)) return fail(RQ_ERR_INVALID_ARG, "codebook formats need LUTs");
   if ((c != nullptr) != (L != nullptr)) return fail(RQ_ERR_INVALID_ARG, "c and L must both be given or both NULL");
+  // 16-level codes are stored sign-magnitude: the GEMM reads the upper half of
+  // the table and takes the lower half as its mirror image
+  auto symmetric16 = [](const uint8_t* lut) {
+    for (int m = 0; m < 8; ++m)
+      if (lut[7 - m] != (uint8_t)(lut[8 + m] | 0x80u)) return false;
+    return true;
+  };
+  if (a_fmt == RQ_LM16 && !symmetric16(a_lut))
+    return fail(RQ_ERR_UNSUPPORTED, "16-level activation table is not symmetric (entry 7-m must be -(entry 8+m))");
+  if (w_fmt == RQ_LM16 && !symmetric16(w_lut))
+    return fail(RQ_ERR_UNSUPPORTED, "16-level weight table is not symmetric (entry 7-m must be -(entry 8+m))");
   if (c && r != 32) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r == 32 (got %d)", r);
   const void* ptrs[] = {a_codes, a_scale, w_codes, w_scale, Y, a_bscale, w_bscale, c, L};
   for (const void* q : ptrs)

@@ -577,7 +577,9 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
           }
         } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
           // code = number of boundaries <= u, read from the cell of u: its
-          // base count plus one compare against the cell's boundary (if any)
+          // base count plus one compare against the cell's boundary (if any);
+          // 16-level codes are stored sign-magnitude (c - 8 above the centre,
+          // (7 - c) | 8 below), both candidates held in the cell
           const float inv = mlt;
           const float cscale = __int_as_float((127 + p.lut_shift) << 23);   // 2^lut_shift
           const float tlo = (float)p.lut_gmin, thi = (float)(p.lut_gmin + p.lut_n - 1) + 0.5f;
@@ -588,9 +590,14 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
             const float t = fminf(fmaxf(__fmul_rn(u, cscale), tlo), thi);   // exact scaling
             const int g = __float_as_int(__fadd_rd(t, 12582912.0f)) - gbias;  // floor(t) - gmin
             const uint2 cell = lut_s[g];
-            const uint32_t c = cell.x + (u >= __uint_as_float(cell.y) ? 1u : 0u);
-            if constexpr (FMT == RQ_FMT_LM16) pk[e >> 3] |= c << (4 * (e & 7));
-            else pk[e >> 4] |= c << (4 * (e & 7) + 2 * ((e >> 3) & 1));   // nibble e%8: elements e%8, e%8+8
+            const bool up = u >= __uint_as_float(cell.y);
+            if constexpr (FMT == RQ_FMT_LM16) {
+              const uint32_t d = (cell.x >> (up ? 8 : 0)) & 0xFu;
+              pk[e >> 3] |= d << (4 * (e & 7));
+            } else {
+              const uint32_t c = cell.x + (up ? 1u : 0u);
+              pk[e >> 4] |= c << (4 * (e & 7) + 2 * ((e >> 3) & 1));   // nibble e%8: elements e%8, e%8+8
+            }
           }
         } else {  // NVFP4: two 16-element groups per lane
           const float inv_t = mlt;
@@ -647,8 +654,11 @@ float e4m3_value(int c) {
 }
 
 // Host: the codebook search table over cells of width 2^-shift, the coarsest
-// grid whose cells hold at most one boundary each.
-bool build_code_lut(K1Params& p, const float* bnd, int nbnd) {
+// grid whose cells hold at most one boundary each.  Entry: the code of the
+// cell's lower part and the cell's boundary (+inf if none); with
+// `sign_magnitude` (16-level codes) the entry holds the stored forms of both
+// codes, lower part in bits 0-7 and upper part in bits 8-15.
+bool build_code_lut(K1Params& p, const float* bnd, int nbnd, bool sign_magnitude) {
   for (int shift = 3; shift <= 14; ++shift) {
     long cell[15];
     bool ok = true;
@@ -668,7 +678,14 @@ bool build_code_lut(K1Params& p, const float* bnd, int nbnd) {
         if (cell[i] < g) ++base;
         if (cell[i] == g) std::memcpy(&b, &bnd[i], 4);
       }
-      p.lut[g - gmin] = make_uint2(base, b);
+      if (sign_magnitude) {
+        // stored form of code c: c - 8 for c >= 8, (7 - c) | 8 below
+        auto sm = [](uint32_t c) { return c >= 8 ? c - 8 : (7 - c) | 8u; };
+        const uint32_t hi = base + 1 <= 15 ? base + 1 : 15;
+        p.lut[g - gmin] = make_uint2(sm(base) | (sm(hi) << 8), b);
+      } else {
+        p.lut[g - gmin] = make_uint2(base, b);
+      }
     }
     return true;
   }
@@ -696,7 +713,7 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
   for (int i = 0; i < 15; ++i) p.bnd[i] = i < a.nbnd ? a.bnd[i] : 0.f;
   p.lut_n = 0;
   if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
-    if (a.nbnd < 1 || !build_code_lut(p, a.bnd, a.nbnd)) return cudaErrorInvalidValue;
+    if (a.nbnd < 1 || !build_code_lut(p, a.bnd, a.nbnd, FMT == RQ_FMT_LM16)) return cudaErrorInvalidValue;
   }
   for (int c = 0; c < 128; ++c) p.rcp_e4m3[c] = (c == 0 || c == 0x7F) ? 0.f : 1.0f / e4m3_value(c);
   const int nblk = a.K / (L * 32);

@@ -83,16 +83,15 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 
-// Eight 4-bit codes (one 32-bit word, code i in bits 4i..4i+3) -> eight LUT
-// bytes: o0 = codes 0-3, o1 = codes 4-7.  prmt reads only the low 16 bits of
-// its selector, so the high codes are shifted down once.
-__device__ __forceinline__ void lut16x8(uint32_t w, const uint32_t (&L)[4], uint32_t& o0, uint32_t& o1) {
-  const uint32_t sel = w & 0x77777777u;
-  const uint32_t sel_hi = sel >> 16;
-  const uint32_t pick = ((w >> 1) & 0x44444444u) | 0x32103210u;
-  const uint32_t pick_hi = pick >> 16;
-  o0 = prmt(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), pick);
-  o1 = prmt(prmt(L[0], L[1], sel_hi), prmt(L[2], L[3], sel_hi), pick_hi);
+// Eight 16-level codes in their stored sign-magnitude form (bits 0-2: distance
+// from the centre, bit 3: lower half) -> eight e4m3 bytes in code order.  The
+// magnitude comes from the 8-entry table of the upper half's centroids (T0, T1);
+// the sign from bit 3, which a sign-replicating permute of the code word (and
+// of the word shifted by 4 for the even nibbles) moves to each byte's sign bit.
+__device__ __forceinline__ void lut_sm8(uint32_t w, uint32_t T0, uint32_t T1, uint32_t& o0, uint32_t& o1) {
+  const uint32_t sel = w & 0x77777777u, w4 = w << 4;
+  o0 = prmt(T0, T1, sel) | (prmt(w4, w, 0xD9C8u) & 0x80808080u);
+  o1 = prmt(T0, T1, sel >> 16) | (prmt(w4, w, 0xFBEAu) & 0x80808080u);
 }
 
 // Sixteen 2-bit codes (one 32-bit word, nibble i holding codes i and i+8 in
@@ -709,7 +708,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
           uint32_t o[8];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) lut16x8(w[j], LA, o[2 * j], o[2 * j + 1]);
+          for (int j = 0; j < 4; ++j) lut_sm8(w[j], LA[2], LA[3], o[2 * j], o[2 * j + 1]);
           const uint32_t rowb = ea + r * 128;
           st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
           st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
@@ -732,7 +731,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             uint32_t o[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) lut16x8(w[j], LW, o[2 * j], o[2 * j + 1]);
+            for (int j = 0; j < 4; ++j) lut_sm8(w[j], LW[2], LW[3], o[2 * j], o[2 * j + 1]);
             const uint32_t rowb = eb + r * 128;
             st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
             st_shared_v4(rowb + (((2 * seg + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);

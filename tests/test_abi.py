@@ -104,10 +104,30 @@ def test_empty_batch_is_a_noop(L):
     assert code == 0, rq.rq_last_error()
     code = L.rq_quantize_weights(rq.LM4, p, 0, 1536, 128, p, p, None, 0, None, p, p, None, None, None)
     assert code == 0, rq.rq_last_error()
-    code = L.rq_w4a4_linear(rq.LM16, rq.LM4, 0, 256, 1536, p, p, None, p, p, None, p, p, None, None, 0, p, 0,
+    # the e4m3 tables are host arrays, read by the argument checks
+    la = np.ascontiguousarray(rq.rq_make_codebook(1536, 16)["centroids_e4m3"], dtype=np.uint8)
+    lw = np.ascontiguousarray(rq.rq_make_codebook(1536, 4)["centroids_e4m3"], dtype=np.uint8)
+    hl = (la.ctypes.data_as(ctypes.c_void_p), lw.ctypes.data_as(ctypes.c_void_p))
+    code = L.rq_w4a4_linear(rq.LM16, rq.LM4, 0, 256, 1536, p, p, None, p, p, None, *hl, None, None, 0, p, 0,
                             None, None)
     assert code == 0, rq.rq_last_error()
     # a negative count is still an error
-    code = L.rq_w4a4_linear(rq.LM16, rq.LM4, -1, 256, 1536, p, p, None, p, p, None, p, p, None, None, 0, p, 0,
+    code = L.rq_w4a4_linear(rq.LM16, rq.LM4, -1, 256, 1536, p, p, None, p, p, None, *hl, None, None, 0, p, 0,
                             None, None)
     assert code == 1
+
+
+def test_codebook_table_must_be_symmetric(L):
+    # 16-level codes are stored sign-magnitude, so the GEMM needs the lower half
+    # of its e4m3 table to mirror the upper half; checked before any launch
+    p = ctypes.c_void_p(0x1000)
+    cb = rq.rq_make_codebook(3072, 16)
+    good = np.ascontiguousarray(cb["centroids_e4m3"], dtype=np.uint8)
+    bad = good.copy()
+    bad[2] ^= 0x01
+    for lut, want in ((good, 0), (bad, 2)):
+        code = L.rq_w4a4_linear(rq.LM16, rq.LM16, 0, 256, 3072, p, p, None, p, p, None,
+                                lut.ctypes.data_as(ctypes.c_void_p), good.ctypes.data_as(ctypes.c_void_p),
+                                None, None, 0, p, 0, None, None)
+        assert code == want, rq.rq_last_error()
+    assert "symmetric" in rq.rq_last_error()

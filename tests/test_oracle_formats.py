@@ -93,3 +93,26 @@ def test_pack_layout():
     c2 = rng.integers(0, 4, size=(3, 64)).astype(np.uint8)
     assert np.array_equal(orc.unpack_crumbs(orc.pack_crumbs(c2)), c2)
     assert list(orc.int4_from_nibble(np.array([0, 7, 8, 9, 15], np.uint8))) == [0, 7, -8, -7, -1]
+
+
+def test_sign_magnitude16_layout():
+    c = np.arange(16, dtype=np.uint8)
+    d = orc.sign_magnitude16(c)
+    # upper half: distance from the centre; lower half: the mirrored distance with bit 3
+    assert list(d) == [15, 14, 13, 12, 11, 10, 9, 8, 0, 1, 2, 3, 4, 5, 6, 7]
+    assert sorted(d) == list(range(16))                                   # a bijection
+    assert np.array_equal(orc.code_from_sign_magnitude16(d), c)
+    q = np.array([[0, 15, 7, 8, 3, 12]], dtype=np.uint8)
+    assert list(orc.pack_nibbles(orc.sign_magnitude16(q))[0]) == [0x7F, 0x08, 0x4C]
+
+
+@pytest.mark.parametrize("K", [1152, 1536, 3072])
+def test_codebook_symmetry_behind_sign_magnitude(K):
+    # the stored form relies on centroid(c) = +-centroid(8 + m): check it on the
+    # FP64 Lloyd-Max solution and on the E4M3 bytes the GEMM multiplies
+    cent, bnd = orc.lloyd_max(K, 16)
+    assert np.allclose(cent[::-1], -cent, rtol=0, atol=1e-12)
+    _, e8 = orc.codebook_tables(K, 16)
+    d = orc.sign_magnitude16(np.arange(16))
+    mag = e8[8 + (d & 7)]
+    assert np.array_equal(e8, np.where(d & 8, mag | 0x80, mag).astype(np.uint8))
