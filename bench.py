@@ -419,7 +419,8 @@ def run_ours(args, w, rank, world, dist):
 # DRAM bytes per launch of the GEMM (read + write) from a 1-pass ncu capture of
 # the current kernels at the full sizes, keyed by workload (the DRAM-traffic
 # summary under profiles/ gives the command and the per-kernel figures).
-TRAFFIC = {"c2": 5_847_552, "c3": 55_207_424, "c4": 56_036_096, "c5": 1_174_680_064}
+# (None: the kernel changed after the last capture)
+TRAFFIC = {"c2": 5_847_552, "c3": None, "c4": 56_036_096, "c5": None}
 
 
 def main():
