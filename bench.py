@@ -5,19 +5,24 @@ One step = the whole online hot path on one batch of tokens:
   K2  rq_w4a4_linear          (4-bit x 4-bit tcgen05 GEMM + fused rank-r low-rank add, BF16 out)
 Weights are folded and quantized once, offline, before timing.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config all|c1..c5] [--impl ours|reference]
 
-Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs the same
-layer on its own token batch (weak scaling, no collective on the data path);
-the time is the max over ranks.  ``--impl reference`` times the CPU oracle on
-the host cores on a bounded sample of the same workload.
+Prints one JSON line (rank 0).  The headline (top-level ``value``, ``roofline``,
+``e2e``, ``cpu_baseline``) is the largest single-GPU layer, the Wan-2.1-like
+W2A4 MLP with CFG (65520 tokens x 1536 -> 8960); with ``--config all`` (the
+default) the other four layers are timed in the same run and reported under
+``configs``.  Multi-GPU (torchrun): every rank runs the same layers on its own
+token batches (weak scaling, no collective on the data path); times are the
+max over ranks.  ``--impl reference`` times the CPU oracle on the host cores on
+a bounded sample of the headline workload.  ``--measure-peaks`` times
+torch._scaled_mm (FP8 e4m3, and block-scaled FP4 where this torch supports it)
+at 8192^3 and prints one JSON line.
 """
 from __future__ import annotations
 
 import argparse
 import dataclasses
 import json
-import math
 import os
 import statistics
 import sys
@@ -32,32 +37,85 @@ sys.path.insert(0, ROOT)
 from rotated_bit_post_b200 import inputs, multirank  # noqa: E402
 
 METRIC = "W4A4 rotated-linear tokens/s & effective TFLOPS (% FP4/FP8 peak) on 1 B200"
+HEADLINE = "c5"
+ORDER = ["c1", "c2", "c3", "c4", "c5"]
 L2_FLUSH_BYTES = 256 << 20
 
+# Dense tensor-core work per SM per clock (FLOP), from the instruction rates:
+# kind::f8f6f4 and kind::i8 retire a 128 x 256 x 32 MMA every 128 cycles
+# (measured back to back on one CTA per SM), the block-scaled FP4 kind twice
+# that (its nominal dense rate is 2x FP8), kind::f16 half of it.
+MMA_FLOP_PER_CLK_SM = {"fp8": 2 * 128 * 256 * 32 / 128, "s8": 2 * 128 * 256 * 32 / 128,
+                       "fp4": 2 * 128 * 256 * 64 / 128, "bf16": 2 * 128 * 256 * 16 / 128}
+NOMINAL_RATIO_TO_BF16 = {"fp8": 2, "s8": 2, "fp4": 4}
 
-def parse():
+# DRAM bytes (read + write) per launch of each kernel from a 1-pass ncu capture
+# of the current kernels at the full sizes; None where the kernel changed after
+# the last capture.  The capture command and per-kernel figures are kept with
+# the other ncu summaries under profiles/.
+TRAFFIC = {
+    "k2": {"c1": None, "c2": None, "c3": None, "c4": None, "c5": None},
+    "k1": {"c1": None, "c2": None, "c3": None, "c4": None, "c5": None},
+}
+
+
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="c2", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--config", default="all", choices=["all"] + ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bf16-linear", action="store_true", help="skip the cuBLAS BF16 linear on the same shapes")
     ap.add_argument("--tokens", type=int, default=0,
                     help="token rows per rank (default: the workload's own); smaller cases for profiler captures")
-    return ap.parse_args()
+    ap.add_argument("--measure-peaks", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="reference arm: CPU seconds for warm-up plus timed steps together")
+    return ap.parse_args(argv)
 
 
-def peaks():
-    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+def measured_peaks():
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+         "source": "fallback"}
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
-        p.update({k: d[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained") if k in d})
+        p.update({k: d[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained", "sm_max_mhz") if k in d})
         p["source"] = "measured"
     return p
+
+
+def tensor_peak(kind: str, sms: int, run_mhz=None):
+    """The denominator for a tensor-core kernel of `kind` ("fp8", "s8", "fp4"):
+    the highest of (a) the measured BF16 matmul burst x the nominal ratio, and
+    (b) the MMA issue rate x SM count x the maximum SM clock.  Both are returned
+    with (c) the issue rate at the clock sampled during the run, for context."""
+    pk = measured_peaks()
+    from_bf16 = pk["bf16_tflops"] * NOMINAL_RATIO_TO_BF16[kind]
+    issue_max = MMA_FLOP_PER_CLK_SM[kind] * sms * pk["sm_max_mhz"] * 1e6 / 1e12
+    peak = max(from_bf16, issue_max)
+    out = {"peak": peak,
+           "peak_source": ("tcgen05 MMA issue rate x %d SMs x %.0f MHz (max clock)" % (sms, pk["sm_max_mhz"])
+                           if issue_max >= from_bf16 else
+                           "%s bf16 burst x nominal ratio %d" % (pk["source"], NOMINAL_RATIO_TO_BF16[kind])),
+           "alt_peaks": {"bf16_burst_x_ratio": from_bf16, "mma_issue_rate_at_max_clock": issue_max}}
+    if run_mhz:
+        out["alt_peaks"]["mma_issue_rate_at_run_clock"] = MMA_FLOP_PER_CLK_SM[kind] * sms * run_mhz * 1e6 / 1e12
+    return out
+
+
+def mma_kind(w):
+    from rotated_bit_post_b200 import rq
+    return "fp4" if w.a_fmt == rq.NVFP4 else "s8" if w.a_fmt == rq.INT4 else "fp8"
+
+
+DTYPE = {"fp4": "e2m1", "s8": "s8", "fp8": "e4m3"}
+DTYPE_NOTE = {"fp4": "e2m1 x e2m1 with UE4M3 block scales, FP32 accumulate",
+              "s8": "INT4 codes as s8 (16 v), S32 accumulate per 128-wide group, FP32 epilogue",
+              "fp8": "codebook codes expanded to e4m3, FP32 accumulate"}
 
 
 def workload_config(w, extra=None):
@@ -74,12 +132,37 @@ def flops_per_step(w):
     return 2.0 * w.M * w.N * w.K + 2.0 * w.M * w.N * w.rank
 
 
+def k1_bytes(w):
+    """Algorithmic bytes of one activation pass: BF16 read, packed codes, the
+    per-token scale, NVFP4 block scales and the BF16 PCA coefficients."""
+    from rotated_bit_post_b200 import rq
+    per_tok = 2 * w.K + w.K // 2 + 4 + (w.K // 16 if w.a_fmt == rq.NVFP4 else 0) + 2 * w.rank
+    return w.M * per_tok
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return int(max(n)) if n else None
+    except Exception:
+        return None
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML while the timed region runs."""
 
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+    PERIOD_S = 0.001
 
     def __init__(self, index):
         self.samples, self.reasons, self.ok = [], set(), False
@@ -104,7 +187,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.005)
+            time.sleep(self.PERIOD_S)
 
     def __enter__(self):
         if self.ok:
@@ -119,7 +202,8 @@ class ClockSampler:
 
     def summary(self):
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, 5 ms period"}
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "nvml, %d ms period, during the timed steps" % int(self.PERIOD_S * 1e3)}
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -132,7 +216,7 @@ def oracle_step(w, X_bits, W_prep, tables):
                               oa["block_scale"], W_prep["block_scale"], ac, wc, oa["coef"], W_prep["coef"])
 
 
-def oracle_setup(w, n_weight_rows=None):
+def oracle_setup(w):
     from oracle import rq_oracle as orc
     sign, perm = orc.make_rotation(w.K, w.block, 0)
     ab = ac = wb = wc = None
@@ -151,46 +235,58 @@ def oracle_setup(w, n_weight_rows=None):
     return W_prep, (sign, perm, ab, ac, wc, U_f32)
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
-        return int(max(n)) if n else os.cpu_count()
-    except Exception:
-        return os.cpu_count()
-
-
-def cpu_baseline(w, target_s=12.0):
-    """Time the oracle (as it stands) on a bounded sample of tokens; tokens/s."""
+def cpu_baseline(w, target_s):
+    """Time the oracle (as it stands) on a bounded sample of tokens; tokens/s.
+    The sample is sized from a doubling probe so that it takes about
+    `target_s` seconds."""
     W_prep, tables = oracle_setup(w)
-    rows = 64
+    oracle_step(w, inputs.activations(w, M=32), W_prep, tables)  # warm (imports, BLAS threads)
+    def timed(n):
+        X = inputs.activations(w, M=n)
+        t0 = time.perf_counter()
+        oracle_step(w, X, W_prep, tables)
+        return time.perf_counter() - t0
+
+    # doubling probes until one takes an eighth of the target (or covers the
+    # layer); the last two separate the per-call cost from the per-token cost
+    n, t_prev = 32, timed(32)
+    while n < w.M:
+        n2 = min(w.M, 2 * n)
+        t2 = timed(n2)
+        per_tok = max((t2 - t_prev) / (n2 - n), t2 / n2 * 1e-3)
+        n, t_prev = n2, t2
+        if t2 >= target_s / 8:
+            break
+    else:
+        per_tok = t_prev / n
+    fixed = max(t_prev - n * per_tok, 0.0)
+    rows = int(min(w.M, max(32, (target_s - fixed) / per_tok)))
+    # a layer smaller than the target is run several times over
+    reps = max(1, int((target_s - fixed) / max(rows * per_tok + fixed, 1e-6))) if rows == w.M else 1
     X = inputs.activations(w, M=rows)
-    oracle_step(w, X, W_prep, tables)  # warm (imports, BLAS threads)
     t0 = time.perf_counter()
-    oracle_step(w, X, W_prep, tables)
+    for _ in range(reps):
+        oracle_step(w, X, W_prep, tables)
     dt = time.perf_counter() - t0
-    rows = int(min(w.M, max(64, rows * target_s / max(dt, 1e-3) / 2)))
-    X = inputs.activations(w, M=rows)
-    t0 = time.perf_counter()
-    oracle_step(w, X, W_prep, tables)
-    dt = time.perf_counter() - t0
-    return {"value": rows / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{rows} of {w.M} tokens of {w.name} (rotate/quantize + FP64 GEMM over all {w.N} outputs), "
-                      f"{dt:.1f} s, weights prepared untimed"}
+    return {"value": rows * reps / dt, "unit": "tokens/s", "cores": host_cores(), "blas_threads": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} x {rows} of {w.M} tokens of {w.name} (rotate/quantize + FP64 GEMM over all {w.N} "
+                      f"outputs), {dt:.1f} s, weights prepared untimed; numpy element-wise steps single-threaded, "
+                      f"FP64 matmul on the BLAS pool"}
 
 
 def run_reference(args, w, rank, world):
     """The oracle as the reference arm: each step is a bounded sample of tokens,
     sized so that warm-up plus timed steps take about two minutes."""
     W_prep, tables = oracle_setup(w)
-    probe = 32
+    probe = 16
     X = inputs.activations(w, M=probe)
     oracle_step(w, X, W_prep, tables)
     t0 = time.perf_counter()
     oracle_step(w, X, W_prep, tables)
     per_row = (time.perf_counter() - t0) / probe
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    rows = int(max(16, min(w.M, budget / max(per_row, 1e-9))))
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)
+    rows = int(max(8, min(w.M, budget / max(per_row, 1e-9))))
     X = inputs.activations(w, M=rows)
     for _ in range(args.warmup):
         oracle_step(w, X, W_prep, tables)
@@ -199,13 +295,13 @@ def run_reference(args, w, rank, world):
         oracle_step(w, X, W_prep, tables)
     dt = time.perf_counter() - t0
     tok_s = rows * args.steps / dt
-    cores = blas_threads()
     out = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic", "config": workload_config(w, {"sample_tokens_per_step": rows}),
            "effective_tflops": flops_per_step(w) * rows / w.M * args.steps / dt / 1e12,
-           "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": host_cores(),
+                            "blas_threads": blas_threads(), "kind": "oracle",
                             "sample": f"{rows} of {w.M} tokens of {w.name} per step (rotate/quantize + FP64 GEMM "
                                       f"over all {w.N} outputs), weights prepared untimed"},
            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -214,225 +310,338 @@ def run_reference(args, w, rank, world):
 
 
 # ----------------------------------------------------------------- GPU arm
-def run_ours(args, w, rank, world, dist):
+class Layer:
+    """One layer on the device: tables, prepared weights, activation buffers and
+    the two hot-path calls through the C ABI."""
+
+    def __init__(self, w, dev, rank, stream):
+        import torch
+        from rotated_bit_post_b200 import rq
+        self.w, self.dev, self.stream, self.rq = w, dev, stream, rq
+        sign, perm, rot = rq.rq_make_rotation(w.K, w.block, 0)
+        self.rot = torch.from_numpy(rot).to(dev)
+        cb_a = rq.rq_make_codebook(w.K, 16) if w.a_fmt == rq.LM16 else None
+        cb_w = cb_a if w.w_fmt == rq.LM16 else (rq.rq_make_codebook(w.K, 4) if w.w_fmt == rq.LM4 else None)
+        self.U = None
+        if w.rank:
+            U_bits, _ = rq.rq_pca_basis(inputs.calibration_tokens(w), w.rank)
+            self.U = torch.from_numpy(U_bits.view(np.int16)).to(dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        Wt = torch.from_numpy(inputs.weights(w).view(np.int16)).to(dev)
+        self.wb = rq.weight_buffers(w.w_fmt, w.N, w.K, w.rank)
+        rq.rq_quantize_weights(w.w_fmt, Wt, w.block, self.rot, None if cb_w is None else cb_w["boundaries_f32"],
+                               self.U, self.wb["L"], self.wb["codes"], self.wb["scale"], self.wb["block_scale"],
+                               self.status)
+        del Wt
+        self.X_np = multirank.rank_activations(w, rank)   # rank r draws its own tokens
+        self.X = torch.from_numpy(self.X_np.view(np.int16)).to(dev)
+        self.ab = rq.act_buffers(w.a_fmt, w.M, w.K, w.rank)
+        self.Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+        self.a_bnd = None if cb_a is None else cb_a["boundaries_f32"]
+        self.a_lut = None if cb_a is None else cb_a["centroids_e4m3"]
+        self.w_lut = None if cb_w is None else cb_w["centroids_e4m3"]
+        self.check()
+
+    def k1(self, x=None):
+        w, ab = self.w, self.ab
+        self.rq.rq_rotate_quantize_act(w.a_fmt, self.X if x is None else x, w.block, self.rot, self.a_bnd, self.U,
+                                       ab["c"], ab["codes"], ab["scale"], ab["block_scale"], self.status,
+                                       self.stream)
+
+    def k2(self, y=None):
+        w, ab, wb = self.w, self.ab, self.wb
+        self.rq.rq_w4a4_linear(w.a_fmt, w.w_fmt, w.M, w.N, w.K, ab["codes"], ab["scale"], ab["block_scale"],
+                               wb["codes"], wb["scale"], wb["block_scale"], self.a_lut, self.w_lut, ab["c"],
+                               wb["L"], self.Y if y is None else y, 0, self.status, self.stream)
+
+    def check(self):
+        import torch
+        torch.cuda.synchronize()
+        rc, code = self.rq.rq_read_status(self.status)
+        if rc != 0:
+            raise RuntimeError(f"kernel status {code:#x}")
+
+
+def time_layer(L, args, flush, dist):
+    """Warm-up, then exactly `steps` timed steps (L2 flushed between them,
+    outside the events); per-step K1 and K2 times from CUDA events on the
+    launching stream.  Returns (k1 ms list, k2 ms list, clock summary)."""
     import torch
-    from rotated_bit_post_b200 import rq
+    stream = L.stream
+    for _ in range(args.warmup):
+        flush.zero_()
+        L.k1()
+        L.k2()
+    L.check()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(L.dev.index) as clocks:
+        for i in range(args.steps):
+            flush.zero_()               # untimed: between the events of consecutive steps
+            ev[i][0].record(stream)
+            L.k1()
+            ev[i][1].record(stream)
+            L.k2()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    L.check()
+    t_k1 = [e[0].elapsed_time(e[1]) for e in ev]
+    t_k2 = [e[1].elapsed_time(e[2]) for e in ev]
+    return t_k1, t_k2, clocks.summary()
+
+
+def time_bf16_linear(L, args, flush):
+    """The same layer as a plain BF16 linear (cuBLAS via torch), for context."""
+    import torch
+    w = L.w
+    Wb = torch.from_numpy(inputs.weights(w).view(np.int16)).to(L.dev).view(torch.bfloat16)
+    Xb = L.X.view(torch.bfloat16)
+    Yb = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=L.dev)
+    for _ in range(3):
+        torch.matmul(Xb, Wb.t(), out=Yb)
+    n_lin = max(5, min(50, args.steps))
+    evl = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_lin)]
+    for a, b in evl:
+        flush.zero_()
+        a.record(L.stream)
+        torch.matmul(Xb, Wb.t(), out=Yb)
+        b.record(L.stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in evl)
+    return {"ms": ms, "tflops": 2.0 * w.M * w.N * w.K / (ms * 1e-3) / 1e12, "tokens_per_s": w.M / (ms * 1e-3),
+            "what": "torch.matmul BF16 x BF16^T (cuBLAS), same M, N, K, L2 flushed before each call, median of "
+                    f"{n_lin}; no rotation or quantization"}
+
+
+def time_e2e(L, args, dist, world):
+    """End to end through the public API with host buffers.  Every step copies
+    its token batch from pinned host memory to the device, runs K1 and K2, and
+    copies its BF16 output back to pinned host memory.  The copies run on their
+    own streams, double-buffered, so that step i+1's upload and step i-1's
+    download overlap step i's kernels (PCIe is full duplex); the timed region
+    spans the first upload to the last download."""
+    import torch
+    w, dev, stream = L.w, L.dev, L.stream
+    X_host = torch.from_numpy(L.X_np.view(np.int16)).pin_memory()
+    Y_host = torch.empty((w.M, w.N), dtype=torch.bfloat16).pin_memory()
+    Xd = [torch.empty_like(L.X), torch.empty_like(L.X)]
+    Yd = [L.Y, torch.empty_like(L.Y)]
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n_e2e = max(5, min(30, args.steps))
+
+    def run_steps(n, e_first=None, e_last=None):
+        up_done = [torch.cuda.Event() for _ in range(n)]
+        x_free = [torch.cuda.Event() for _ in range(n)]
+        comp_done = [torch.cuda.Event() for _ in range(n)]
+        down_done = [torch.cuda.Event() for _ in range(n)]
+        if e_first is not None:
+            e_first.record(s_up)
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(x_free[i - 2])
+                Xd[b].copy_(X_host, non_blocking=True)
+                up_done[i].record(s_up)
+            stream.wait_event(up_done[i])
+            if i >= 2:
+                stream.wait_event(down_done[i - 2])
+            L.k1(Xd[b])
+            x_free[i].record(stream)
+            L.k2(Yd[b])
+            comp_done[i].record(stream)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(comp_done[i])
+                Y_host.copy_(Yd[b], non_blocking=True)
+                down_done[i].record(s_down)
+        if e_last is not None:
+            e_last.record(s_down)
+
+    run_steps(3)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    run_steps(n_e2e, e0, e1)
+    torch.cuda.synchronize()
+    ms = multirank.max_over_ranks(dist, e0.elapsed_time(e1) / n_e2e, dev)
+    L.check()
+    return {"value": multirank.aggregate_tokens_per_s(w.M, world, ms), "unit": "tokens/s",
+            "h2d_bytes_per_step": L.X.numel() * 2, "d2h_bytes_per_step": L.Y.numel() * 2, "ms_per_step": ms,
+            "steps": n_e2e,
+            "note": "per step: pinned host X -> device, K1, K2, device Y -> pinned host; uploads and downloads "
+                    "on their own streams overlap the neighbouring steps' kernels"}
+
+
+def layer_result(L, args, t_k1, t_k2, clocks, dist, world, sms):
+    """Per-layer figures: step time (sum over exactly `steps` steps, max over
+    ranks), per-kernel medians, and the roofline of the dominant kernel."""
+    w = L.w
+    step_ms_total = multirank.max_over_ranks(dist, sum(a + b for a, b in zip(t_k1, t_k2)), L.dev)
+    ms_per_step = step_ms_total / args.steps
+    med_step = statistics.median(a + b for a, b in zip(t_k1, t_k2))
+    k1_ms, k2_ms = statistics.median(t_k1), statistics.median(t_k2)
+    fl = flops_per_step(w)
+    kind = mma_kind(w)
+    tp = tensor_peak(kind, sms, clocks.get("sm_mhz"))
+    pk = measured_peaks()
+    k2_tflops = fl / (k2_ms * 1e-3) / 1e12
+    kb = k1_bytes(w)
+    k1_gbs = kb / (k1_ms * 1e-3) / 1e9
+    k1_roof = {"kernel": "k1_rotate_quantize (rq_rotate_quantize_act)", "bound": "hbm", "achieved": k1_gbs,
+               "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": k1_gbs / pk["hbm_gbs"],
+               "frac_of_8tbs": k1_gbs / 8000.0,
+               "peak_source": pk["source"] + " copy (MEASURED_PEAKS hbm_gbs)",
+               "algorithmic_per_launch": f"{kb} B (2K + K/2 + 4 [+ K/16] [+ 2r] per token)",
+               "traffic": None if args.tokens else TRAFFIC["k1"].get(w.name)}
+    k2_roof = {"kernel": "gemm kernel of rq_w4a4_linear", "bound": "tensor", "achieved": k2_tflops,
+               "peak": tp["peak"], "unit": "TFLOP/s", "frac": k2_tflops / tp["peak"],
+               "peak_source": tp["peak_source"], "alt_peaks": tp["alt_peaks"],
+               "algorithmic_per_launch": f"{fl:.4g} FLOP (2MNK + 2MNr)",
+               "traffic": None if args.tokens else TRAFFIC["k2"].get(w.name)}
+    dominant = k2_roof if k2_ms >= k1_ms else k1_roof
+    return {
+        "config": workload_config(w),
+        "dtype": DTYPE[kind], "dtype_note": DTYPE_NOTE[kind],
+        "tokens_per_s": multirank.aggregate_tokens_per_s(w.M, world, ms_per_step),
+        "ms_per_step": ms_per_step, "median_ms_per_step": med_step,
+        "effective_tflops": fl * world / (ms_per_step * 1e-3) / 1e12,
+        "effective_frac_of_peak": fl / (med_step * 1e-3) / 1e12 / tp["peak"],
+        "kernels": {"k1_rotate_quantize_us": 1e3 * k1_ms, "k1_gbs": k1_gbs, "k1_frac_hbm": k1_gbs / pk["hbm_gbs"],
+                    "k2_gemm_us": 1e3 * k2_ms, "k2_tflops": k2_tflops, "k2_frac_peak": k2_tflops / tp["peak"],
+                    "timing": "medians of the per-step CUDA-event times"},
+        "roofline": dominant, "roofline_k1": k1_roof, "roofline_k2": k2_roof,
+        "clocks": clocks,
+    }
+
+
+def run_ours(args, names, rank, world, dist):
+    import torch
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-
-    # ---------------- offline preparation (untimed)
-    sign, perm, rot = rq.rq_make_rotation(w.K, w.block, 0)
-    rot_t = torch.from_numpy(rot).to(dev)
-    cb_a = rq.rq_make_codebook(w.K, 16) if w.a_fmt == rq.LM16 else None
-    cb_w = cb_a if w.w_fmt == rq.LM16 else (rq.rq_make_codebook(w.K, 4) if w.w_fmt == rq.LM4 else None)
-    U_t = None
-    if w.rank:
-        U_bits, _ = rq.rq_pca_basis(inputs.calibration_tokens(w), w.rank)
-        U_t = torch.from_numpy(U_bits.view(np.int16)).to(dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    Wt = torch.from_numpy(inputs.weights(w).view(np.int16)).to(dev)
-    wb = rq.weight_buffers(w.w_fmt, w.N, w.K, w.rank)
-    rq.rq_quantize_weights(w.w_fmt, Wt, w.block, rot_t, None if cb_w is None else cb_w["boundaries_f32"], U_t,
-                           wb["L"], wb["codes"], wb["scale"], wb["block_scale"], status)
-    del Wt
-    # this rank's token batch (rank r draws its own tokens)
-    X_np = multirank.rank_activations(w, rank)
-    X = torch.from_numpy(X_np.view(np.int16)).to(dev)
-    ab = rq.act_buffers(w.a_fmt, w.M, w.K, w.rank)
-    Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
-    a_bnd = None if cb_a is None else cb_a["boundaries_f32"]
-    a_lut = None if cb_a is None else cb_a["centroids_e4m3"]
-    w_lut = None if cb_w is None else cb_w["centroids_e4m3"]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def k1(x):
-        rq.rq_rotate_quantize_act(w.a_fmt, x, w.block, rot_t, a_bnd, U_t, ab["c"], ab["codes"], ab["scale"],
-                                  ab["block_scale"], status, stream)
-
-    def k2(y=None):
-        rq.rq_w4a4_linear(w.a_fmt, w.w_fmt, w.M, w.N, w.K, ab["codes"], ab["scale"], ab["block_scale"],
-                          wb["codes"], wb["scale"], wb["block_scale"], a_lut, w_lut, ab["c"], wb["L"],
-                          Y if y is None else y, 0, status, stream)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        k1(X)
-        k2()
-    torch.cuda.synchronize()
-    rc, code = rq.rq_read_status(status)
-    if rc != 0:
-        raise RuntimeError(f"kernel status {code:#x}")
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
-        for i in range(args.steps):
-            flush.zero_()               # untimed: between the events of consecutive steps
-            ev[i][0].record(stream)
-            k1(X)
-            ev[i][1].record(stream)
-            k2()
-            ev[i][2].record(stream)
-        torch.cuda.synchronize()
-    barrier()
-    t_k1 = [e[0].elapsed_time(e[1]) for e in ev]
-    t_k2 = [e[1].elapsed_time(e[2]) for e in ev]
-    step_ms = sum(a + b for a, b in zip(t_k1, t_k2))
-    step_ms = multirank.max_over_ranks(dist, step_ms, dev)
-    rc, code = rq.rq_read_status(status)
-    if rc != 0:
-        raise RuntimeError(f"kernel status {code:#x}")
-
-    # ---------------- the same layer as a plain BF16 linear (cuBLAS via torch), for context
-    bf16_linear = None
-    if not args.no_bf16_linear:
-        Wb = torch.from_numpy(inputs.weights(w).view(np.int16)).to(dev).view(torch.bfloat16)
-        Xb = X.view(torch.bfloat16)
-        Yb = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
-        for _ in range(3):
-            torch.matmul(Xb, Wb.t(), out=Yb)
-        n_lin = max(5, min(50, args.steps))
-        evl = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_lin)]
-        for a, b in evl:
-            flush.zero_()
-            a.record(stream)
-            torch.matmul(Xb, Wb.t(), out=Yb)
-            b.record(stream)
-        torch.cuda.synchronize()
-        lin_ms = statistics.mean(a.elapsed_time(b) for a, b in evl)
-        bf16_linear = {"ms": lin_ms, "tflops": 2.0 * w.M * w.N * w.K / (lin_ms * 1e-3) / 1e12,
-                       "tokens_per_s": w.M / (lin_ms * 1e-3), "what": "torch.matmul BF16 x BF16^T (cuBLAS), "
-                       "same M, N, K, L2 flushed before each call, no rotation or quantization"}
-        del Wb, Yb
-
-    # ---------------- end to end through the public API with host buffers
-    # Every step copies its token batch from pinned host memory to the device,
-    # runs K1 and K2, and copies its BF16 output back to pinned host memory.
-    # The copies run on their own streams, double-buffered, so that step i+1's
-    # upload and step i-1's download overlap step i's kernels (PCIe is full
-    # duplex); the timed region spans the first upload to the last download.
-    e2e = None
-    if not args.no_e2e:
-        X_host = torch.from_numpy(X_np.view(np.int16)).pin_memory()
-        Y_host = torch.empty((w.M, w.N), dtype=torch.bfloat16).pin_memory()
-        Xd = [torch.empty_like(X), torch.empty_like(X)]
-        Yd = [Y, torch.empty_like(Y)]
-        s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        n_e2e = max(5, min(50, args.steps))
-
-        def run_steps(n, e_first=None, e_last=None):
-            up_done = [torch.cuda.Event() for _ in range(n)]
-            x_free = [torch.cuda.Event() for _ in range(n)]
-            comp_done = [torch.cuda.Event() for _ in range(n)]
-            down_done = [torch.cuda.Event() for _ in range(n)]
-            if e_first is not None:
-                e_first.record(s_up)
-            for i in range(n):
-                b = i & 1
-                with torch.cuda.stream(s_up):
-                    if i >= 2:
-                        s_up.wait_event(x_free[i - 2])
-                    Xd[b].copy_(X_host, non_blocking=True)
-                    up_done[i].record(s_up)
-                stream.wait_event(up_done[i])
-                if i >= 2:
-                    stream.wait_event(down_done[i - 2])
-                k1(Xd[b])
-                x_free[i].record(stream)
-                k2(Yd[b])
-                comp_done[i].record(stream)
-                with torch.cuda.stream(s_down):
-                    s_down.wait_event(comp_done[i])
-                    Y_host.copy_(Yd[b], non_blocking=True)
-                    down_done[i].record(s_down)
-            if e_last is not None:
-                e_last.record(s_down)
-
-        run_steps(3)
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        run_steps(n_e2e, e0, e1)
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        e2e_ms = multirank.max_over_ranks(dist, e2e_ms, dev)
-        rc, code = rq.rq_read_status(status)
-        if rc != 0:
-            raise RuntimeError(f"kernel status {code:#x}")
-        e2e = {"value": multirank.aggregate_tokens_per_s(w.M, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": X.numel() * 2,
-               "d2h_bytes_per_step": Y.numel() * 2, "ms_per_step": e2e_ms,
-               "note": "per step: pinned host X -> device, K1, K2, device Y -> pinned host; uploads and "
-                       "downloads on their own streams overlap the neighbouring steps' kernels"}
-        del Xd, Yd
+    results = {}
+    for name in names:
+        w = inputs.WORKLOADS[name]
+        if args.tokens:
+            w = dataclasses.replace(w, M=args.tokens)
+        L = Layer(w, dev, rank, stream)
+        t_k1, t_k2, clocks = time_layer(L, args, flush, dist)
+        res = layer_result(L, args, t_k1, t_k2, clocks, dist, world, sms)
+        if not args.no_bf16_linear:
+            res["bf16_linear"] = time_bf16_linear(L, args, flush)
+            res["speedup_vs_bf16_linear"] = res["bf16_linear"]["ms"] / res["median_ms_per_step"]
+        if not args.no_e2e:
+            res["e2e"] = time_e2e(L, args, dist, world)
+        results[name] = res
+        del L
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return
-
-    ms_per_step = step_ms / args.steps
-    k1_ms = statistics.mean(t_k1)
-    k2_ms = statistics.mean(t_k2)
-    tok_s = multirank.aggregate_tokens_per_s(w.M, world, ms_per_step)
-    fl = flops_per_step(w)
-    pk = peaks()
-    mma_ratio = 4 if w.a_fmt == rq.NVFP4 else 2          # nominal FP4 / FP8 vs BF16 dense ratio
-    tensor_peak = pk["bf16_tflops"] * mma_ratio
-    k2_tflops = fl / (k2_ms * 1e-3) / 1e12
-    k1_bytes = w.M * (2 * w.K + w.K // 2 + 4 + (w.K // 16 if w.a_fmt == rq.NVFP4 else 0) + 2 * w.rank)
-    k1_gbs = k1_bytes / (k1_ms * 1e-3) / 1e9
-    dominant_is_k2 = k2_ms >= k1_ms
-    if dominant_is_k2:
-        roof = {"kernel": "rq_w4a4_linear (gemm_fp8/nvf4)", "bound": "tensor", "achieved": k2_tflops,
-                "peak": tensor_peak, "unit": "TFLOP/s", "frac": k2_tflops / tensor_peak,
-                "peak_source": f"{pk['source']} bf16 burst {pk['bf16_tflops']} x nominal ratio {mma_ratio} "
-                               f"({'fp4' if mma_ratio == 4 else 'fp8'}/bf16)",
-                "algorithmic_per_launch": f"{fl:.4g} FLOP (2MNK + 2MNr)", "traffic": None if args.tokens else TRAFFIC.get(w.name)}
-    else:
-        roof = {"kernel": "rq_rotate_quantize_act", "bound": "hbm", "achieved": k1_gbs, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": k1_gbs / pk["hbm_gbs"], "peak_source": pk["source"] + " copy",
-                "algorithmic_per_launch": f"{k1_bytes} B", "traffic": None}
-    out = {"metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "e4m3" if w.a_fmt != rq.NVFP4 else "e2m1",
+    head = results[HEADLINE] if HEADLINE in results else results[names[-1]]
+    hw = inputs.WORKLOADS[HEADLINE if HEADLINE in results else names[-1]]
+    out = {"metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+           "median_ms_per_step": head["median_ms_per_step"], "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": head["dtype"], "dtype_note": head["dtype_note"],
            "data": "synthetic (seeded DiT-shaped activations, N(0,0.02) weights)",
-           "config": workload_config(w, {"parallelism": f"token-parallel x{world} (independent batches)"}),
-           "effective_tflops": fl * world / (ms_per_step * 1e-3) / 1e12,
-           "effective_frac_of_peak": fl / (ms_per_step * 1e-3) / 1e12 / tensor_peak,
-           "kernels": {"k1_rotate_quantize_us": 1e3 * k1_ms, "k1_gbs": k1_gbs,
-                       "k1_frac_hbm": k1_gbs / pk["hbm_gbs"], "k2_gemm_us": 1e3 * k2_ms,
-                       "k2_tflops": k2_tflops, "k2_frac_peak": k2_tflops / tensor_peak},
-           "roofline": roof, "clocks": clocks.summary(), "e2e": e2e,
-           "bf16_linear": bf16_linear,
-           "speedup_vs_bf16_linear": None if bf16_linear is None else bf16_linear["ms"] / ms_per_step,
-           "gpu_launches": 2 * args.steps}
+           "config": dict(head["config"], parallelism=f"token-parallel x{world} (independent batches)"),
+           "effective_tflops": head["effective_tflops"], "effective_frac_of_peak": head["effective_frac_of_peak"],
+           "kernels": head["kernels"], "roofline": head["roofline"], "clocks": head["clocks"],
+           "e2e": head.get("e2e"), "bf16_linear": head.get("bf16_linear"),
+           "speedup_vs_bf16_linear": head.get("speedup_vs_bf16_linear"),
+           "gpu_launches": 2 * args.steps,
+           "gpu_launches_note": "per timed step of the headline layer: one K1 and one K2 launch"}
+    if len(names) > 1:
+        out["configs"] = {n: results[n] for n in names}
     if not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w)
+        out["cpu_baseline"] = cpu_baseline(hw, 15.0)
+        if len(names) > 1:
+            for n in names:
+                if n != HEADLINE:
+                    out["configs"][n]["cpu_baseline"] = cpu_baseline(inputs.WORKLOADS[n], 3.0)
+            out["configs"][HEADLINE]["cpu_baseline"] = out["cpu_baseline"]
     print(json.dumps(out), flush=True)
 
 
-# DRAM bytes per launch of the GEMM (read + write) from a 1-pass ncu capture of
-# the current kernels at the full sizes, keyed by workload (the DRAM-traffic
-# summary under profiles/ gives the command and the per-kernel figures).
-# (None: the kernel changed after the last capture)
-TRAFFIC = {"c2": 5_847_552, "c3": None, "c4": 56_036_096, "c5": None}
+# ----------------------------------------------------------------- peaks
+def measure_peaks():
+    """torch._scaled_mm at 8192^3: FP8 e4m3 (per-tensor scales) and, where this
+    torch supports it, NVFP4 (e2m1 with e4m3 scales per 16 elements); best of
+    10 calls (burst) and back to back for 4 s (sustained)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    n = 8192
+    out = {"what": "torch._scaled_mm %d^3" % n, "torch": torch.__version__}
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        best = 1e9
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            best = min(best, a.elapsed_time(b))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cnt = 0
+        t0 = time.time()
+        with ClockSampler(0) as clk:
+            a.record()
+            while time.time() - t0 < 4.0:
+                for _ in range(20):
+                    fn()
+                cnt += 20
+                torch.cuda.synchronize()
+            b.record()
+            torch.cuda.synchronize()
+        sus = a.elapsed_time(b) / cnt
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12, 2.0 * n ** 3 / (sus * 1e-3) / 1e12, clk.summary()
+
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    burst, sus, clk = timed(lambda: torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16))
+    out["fp8_e4m3"] = {"burst_tflops": burst, "sustained_tflops": sus, "clocks": clk}
+    try:
+        fp4 = getattr(torch, "float4_e2m1fn_x2")
+        a4 = torch.randint(0, 256, (n, n // 2), dtype=torch.uint8, device=dev).view(fp4)
+        b4 = torch.randint(0, 256, (n, n // 2), dtype=torch.uint8, device=dev).view(fp4)
+        # block scales: one e4m3 per 16 elements, in the swizzled 128x4 layout cuBLAS expects
+        sa = torch.full((n * n // 16,), 1.0, device=dev).to(torch.float8_e4m3fn)
+        sb = torch.full((n * n // 16,), 1.0, device=dev).to(torch.float8_e4m3fn)
+        burst, sus, clk = timed(lambda: torch._scaled_mm(a4, b4.t(), sa, sb, out_dtype=torch.bfloat16))
+        out["fp4_nvfp4"] = {"burst_tflops": burst, "sustained_tflops": sus, "clocks": clk}
+    except Exception as e:  # not every torch build routes block-scaled FP4 through _scaled_mm
+        out["fp4_nvfp4"] = {"unavailable": f"{type(e).__name__}: {str(e)[:200]}"}
+    print(json.dumps(out), flush=True)
 
 
 def main():
     args = parse()
-    w = inputs.WORKLOADS[args.config]
-    if args.tokens:
-        w = dataclasses.replace(w, M=args.tokens)
+    if args.measure_peaks:
+        measure_peaks()
+        return
+    names = ORDER if args.config == "all" else [args.config]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
-        # the CPU oracle runs once, on rank 0; other ranks have nothing to do
+        # the CPU oracle runs once, on rank 0, on the headline layer; other ranks have nothing to do
         if rank == 0:
+            w = inputs.WORKLOADS[HEADLINE if args.config == "all" else args.config]
+            if args.tokens:
+                w = dataclasses.replace(w, M=args.tokens)
             run_reference(args, w, rank, world)
         return
     dist = None
@@ -444,7 +653,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(args, w, rank, world, dist)
+        run_ours(args, names, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()
