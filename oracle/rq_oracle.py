@@ -27,7 +27,8 @@ Readings taken where the pages are silent:
 FP32 arithmetic with round-to-nearest-even and no fused multiply-add except
 where a product is exact; butterfly stages in ascending stride; a perfect
 pairwise sum of squares inside each block and a sequential sum over blocks;
-sequential dot products for the PCA coefficients; signs applied before the
+the PCA coefficients summed per 128-channel chunk in k order, chunks added in
+order, the residual subtracted in order of j; signs applied before the
 permutation; SplitMix64 for the rotation's random draws.
 
 Parity status of each function is stated in its docstring ("pinned by ...").
@@ -189,8 +190,10 @@ def e4m3_encode(a: np.ndarray) -> np.ndarray:
     The sign bit is kept for negative inputs, -0.0 included.
 
     Pinned by: grid facts of the OCP definition (max 448, min subnormal 2^-9,
-    ties to even mantissa) in tests/test_oracle_formats.py and by the GPU
-    conversion instruction over sampled FP32 patterns (tests/test_gpu_formats.py)."""
+    ties to even mantissa) and torch's float8_e4m3fn cast in
+    tests/test_oracle_formats.py, and by the GPU's cvt.rn.satfinite.e4m3x2.f32
+    over FP32 patterns spanning the format's range, every midpoint +-1 ulp and
+    the saturation edges (tests/test_gpu_formats.py)."""
     a = np.asarray(a, dtype=np.float32)
     code = _grid_round(a, E4M3_GRID).astype(np.uint8)
     return code | np.where(np.signbit(a), np.uint8(0x80), np.uint8(0))
@@ -204,7 +207,9 @@ def e4m3_decode(code: np.ndarray) -> np.ndarray:
 
 def e2m1_encode(a: np.ndarray) -> np.ndarray:
     """FP32 -> E2M1 nibble (sign in bit 3), round to nearest even, saturating to
-    +-6.  Pinned like ``e4m3_encode``."""
+    +-6.  Pinned by the grid, tie and saturation cases and a brute-force
+    nearest-value search in tests/test_oracle_formats.py, and by the GPU's
+    cvt.rn.satfinite.e2m1x2.f32 (tests/test_gpu_formats.py)."""
     a = np.asarray(a, dtype=np.float32)
     code = _grid_round(a, E2M1_GRID).astype(np.uint8)
     return code | np.where(np.signbit(a), np.uint8(8), np.uint8(0))
@@ -319,8 +324,8 @@ def pca_basis(calib_f32: np.ndarray, r: int):
     activation variance via PCA).  FP64; sign fixed so that the largest-magnitude
     entry of each vector is positive.  Returns (U float64 K x r, eigenvalues r).
 
-    Pinned by: U^T U = I, the eigen-equation residual and descending order
-    (tests/test_oracle_pca.py)."""
+    Pinned by: U^T U = I, the eigen-equation residual, descending order and
+    the sign rule (tests/test_oracle_quant.py::test_pca_basis)."""
     X = calib_f32.astype(np.float64)
     S = X.T @ X / X.shape[0]
     w, V = np.linalg.eigh(S)
@@ -331,21 +336,50 @@ def pca_basis(calib_f32: np.ndarray, r: int):
     return V, w
 
 
+PROJ_CHUNK = 128
+
+
 def project_coefficients(x_f32: np.ndarray, U_f32: np.ndarray) -> np.ndarray:
-    """c = x U in FP32, each c_j accumulated sequentially over k = 0..K-1 (every
-    product of two BF16 values is exact in FP32, so this is the FP32 dot product
-    in natural order), returned as FP32 values before BF16 rounding."""
+    """c = x U in FP32 (DiRotQ abstract: the coefficients of the activation in
+    the PCA subspace), returned as FP32 values before their BF16 rounding.
+
+    Reading of the summation order (the pages fix none): the K input channels
+    are cut into chunks of 128 consecutive channels; inside a chunk the
+    products x_k U_kj are added one after another in natural k order, starting
+    from the first product; the chunk partials are then added in chunk order,
+    starting from chunk 0.  Every product of two BF16 values is exact in FP32
+    (16 significant bits; magnitudes here stay far from the FP32 subnormal
+    range), so "add the product" and "fused multiply-add" give the same value.
+    K must be a multiple of 128.
+
+    Pinned by: tests/test_oracle_quant.py (an element-by-element float32 loop
+    restating this order; inputs on which a BLAS product, a pairwise order, a
+    single sequential chain and a 64-wide chunking all give other values)."""
     M, K = x_f32.shape
-    acc = np.zeros((M, U_f32.shape[1]), dtype=F32)
-    for k in range(K):
-        acc = acc + x_f32[:, k:k + 1] * U_f32[k:k + 1, :]
-    return acc
+    if K % PROJ_CHUNK:
+        raise ValueError("the projection needs K % 128 == 0")
+    r = U_f32.shape[1]
+    x = x_f32.astype(F32)
+    U = U_f32.astype(F32)
+    total = None
+    for t in range(K // PROJ_CHUNK):
+        part = np.zeros((M, r), dtype=F32)
+        for k in range(t * PROJ_CHUNK, (t + 1) * PROJ_CHUNK):
+            part = part + x[:, k:k + 1] * U[k:k + 1, :]
+        total = part if total is None else total + part
+    return total
 
 
 def residual(x_f32: np.ndarray, c_f32: np.ndarray, U_f32: np.ndarray) -> np.ndarray:
-    """x_res[k] = x[k] - sum_j c_j U[k, j], subtracting the (exact) products in
-    order j = 0..r-1 in FP32 (DiRotQ abstract: the components outside the PCA
-    subspace are the ones quantized to 4 bit)."""
+    """x_res[k] = x[k] - sum_j c_j U[k, j] (DiRotQ abstract: the components
+    outside the PCA subspace are the ones quantized to 4 bit), with c the
+    BF16-rounded coefficients: starting from x[k], the exact products c_j U[k, j]
+    are subtracted one after another in order j = 0..r-1, each subtraction
+    rounded to FP32.
+
+    Pinned by: tests/test_oracle_quant.py (a float32 loop restating the order;
+    inputs on which a BLAS product, the reverse order of j and unrounded
+    coefficients give other values)."""
     xr = x_f32.astype(F32).copy()
     for j in range(U_f32.shape[1]):
         xr = xr - c_f32[:, j:j + 1] * U_f32[None, :, j]

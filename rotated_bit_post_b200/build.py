@@ -20,7 +20,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "librq.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["rq_api.cu", "rq_k1.cu", "rq_k2.cu", "rq_host.cpp"]
+SOURCES = ["rq_api.cu", "rq_k1.cu", "rq_k2.cu", "rq_host.cpp", "rq_check.cu"]
 HEADERS = ["rq_ptx.cuh", "rq_internal.h", "rq_host.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -41,7 +41,7 @@ def _flags(verbose_ptxas: bool):
 def _stale(obj: str, src: str) -> bool:
     if not os.path.exists(obj):
         return True
-    deps = [src] + [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "rq.h"), __file__]
+    deps = [src] + [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, h) for h in os.listdir(INCLUDE)] + [__file__]
     t = os.path.getmtime(obj)
     return any(os.path.getmtime(d) > t for d in deps)
 

@@ -271,36 +271,55 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
 
     if constexpr (PROJ) {
       // ---------------------------------------------------------- coefficients
-      // c[row][j] = bf16(sum_k x[row][k] U[k][j]), each sum one sequential FP32
-      // chain in k, read straight from the BF16 rows as they landed.  Warp w
-      // takes rows w and w + 16 (two interleaved chains), lane j the column j.
-      // fma.rn.f32.bf16 rounds the exact product plus the addend once, like
-      // an FMA on the widened operands.
-      if (warp < nr) {
-        const bool two = warp + 16 < nr;
-        const uint4* uj = reinterpret_cast<const uint4*>(ut + (size_t)lane * ut_pitch(K));
-        const uint4* xa = reinterpret_cast<const uint4*>(land + (size_t)warp * K);
-        const uint4* xb = reinterpret_cast<const uint4*>(land + (size_t)(two ? warp + 16 : warp) * K);
-        float ca = 0.f, cb = 0.f;
-#pragma unroll 2
-        for (int k8 = 0; k8 < K / 8; ++k8) {
-          const uint4 u = uj[k8], a = xa[k8], b = xb[k8];
-          ca = fma_bf16<0, 0>(a.x, u.x, ca); cb = fma_bf16<0, 0>(b.x, u.x, cb);
-          ca = fma_bf16<1, 1>(a.x, u.x, ca); cb = fma_bf16<1, 1>(b.x, u.x, cb);
-          ca = fma_bf16<0, 0>(a.y, u.y, ca); cb = fma_bf16<0, 0>(b.y, u.y, cb);
-          ca = fma_bf16<1, 1>(a.y, u.y, ca); cb = fma_bf16<1, 1>(b.y, u.y, cb);
-          ca = fma_bf16<0, 0>(a.z, u.z, ca); cb = fma_bf16<0, 0>(b.z, u.z, cb);
-          ca = fma_bf16<1, 1>(a.z, u.z, ca); cb = fma_bf16<1, 1>(b.z, u.z, cb);
-          ca = fma_bf16<0, 0>(a.w, u.w, ca); cb = fma_bf16<0, 0>(b.w, u.w, cb);
-          ca = fma_bf16<1, 1>(a.w, u.w, ca); cb = fma_bf16<1, 1>(b.w, u.w, cb);
+      // c[row][j] = bf16(sum_k x[row][k] U[k][j]) with the sum cut into
+      // 128-wide chunks of k: inside a chunk one sequential FP32 chain in k
+      // order, read straight from the BF16 rows as they landed; the chunk sums
+      // are then added in chunk order.  fma.rn.f32.bf16 rounds the exact product
+      // plus the running sum once, like an add of the (exact) product.  Lane j
+      // takes column j; a warp takes units of four rows of one chunk (four
+      // independent chains sharing each U^T load).  The chunk sums go to the
+      // lower half of the FP32 row buffer, unused until the rows are widened.
+      {
+        const int nch = K / 128;
+        const int RG = (nr + 3) >> 2;
+        float* cpart = xf;   // [nr][nch][32]
+        for (int gi = warp; gi < RG * nch; gi += K1_WARPS) {
+          const int t = gi / RG, rb = (gi - t * RG) * 4;
+          const uint4* uj = reinterpret_cast<const uint4*>(ut + (size_t)lane * ut_pitch(K) + t * 128);
+          const uint4* xr[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            xr[i] = reinterpret_cast<const uint4*>(land + (size_t)min(rb + i, nr - 1) * K + t * 128);
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+          for (int k8 = 0; k8 < 16; ++k8) {
+            const uint4 u = uj[k8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 a = xr[i][k8];
+              acc[i] = fma_bf16<0, 0>(a.x, u.x, acc[i]);
+              acc[i] = fma_bf16<1, 1>(a.x, u.x, acc[i]);
+              acc[i] = fma_bf16<0, 0>(a.y, u.y, acc[i]);
+              acc[i] = fma_bf16<1, 1>(a.y, u.y, acc[i]);
+              acc[i] = fma_bf16<0, 0>(a.z, u.z, acc[i]);
+              acc[i] = fma_bf16<1, 1>(a.z, u.z, acc[i]);
+              acc[i] = fma_bf16<0, 0>(a.w, u.w, acc[i]);
+              acc[i] = fma_bf16<1, 1>(a.w, u.w, acc[i]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (rb + i < nr) cpart[((size_t)(rb + i) * nch + t) * 32 + lane] = acc[i];
         }
-        const uint16_t ha = __bfloat16_as_ushort(__float2bfloat16_rn(ca));
-        p.coef[(size_t)(r0 + warp) * 32 + lane] = ha;
-        negc[warp * 32 + lane] = -bf16_bits_to_f32(ha);
-        if (two) {
-          const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(cb));
-          p.coef[(size_t)(r0 + warp + 16) * 32 + lane] = hb;
-          negc[(warp + 16) * 32 + lane] = -bf16_bits_to_f32(hb);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < nr * 32; idx += K1_THREADS) {
+          const int row = idx >> 5, j = idx & 31;
+          const float* cp = cpart + (size_t)row * nch * 32 + j;
+          float s = cp[0];
+          for (int t = 1; t < nch; ++t) s = __fadd_rn(s, cp[t * 32]);
+          const uint16_t h = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+          p.coef[(size_t)(r0 + row) * 32 + j] = h;
+          negc[row * 32 + j] = -bf16_bits_to_f32(h);
         }
       }
       __syncthreads();

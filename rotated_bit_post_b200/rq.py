@@ -1,4 +1,5 @@
-"""Python binding of the C ABI in include/rq.h (argument marshalling only).
+"""Python binding of the C ABI in include/rq.h and include/rq_check.h (argument
+marshalling only).
 
 Every function keeps the C name.  Device buffers are torch CUDA tensors (their
 data pointers are passed through); host tables are numpy arrays.  All compute
@@ -36,6 +37,8 @@ SIGNATURES = [
       _c_i32, _c_p, _c_i32, _c_p, _c_p]),
     ("rq_read_status", _c_i32, [_c_p, _c_p, _c_p]),
     ("rq_last_error", ctypes.c_char_p, []),
+    # include/rq_check.h
+    ("rq_convert_check", _c_i32, [_c_p, _c_i32, _c_p, _c_p, _c_p]),
 ]
 
 
@@ -157,6 +160,13 @@ def rq_read_status(status, stream=None):
     if rc not in (0, 5):
         _check("rq_read_status", rc)
     return rc, code.value
+
+
+def rq_convert_check(x, e4m3_out, e2m1_out, stream=None):
+    """E4M3 bytes and E2M1 nibbles of the FP32 device tensor x, from the
+    hardware conversions the activation kernel uses (include/rq_check.h)."""
+    _check("rq_convert_check", lib().rq_convert_check(_dev(x), x.numel(), _dev(e4m3_out), _dev(e2m1_out),
+                                                      _stream(stream)))
 
 
 def rq_last_error() -> str:

@@ -1,5 +1,5 @@
-"""The C-ABI library: it loads without a GPU, exports every symbol include/rq.h
-declares, its host-side preparation agrees with the oracle, and argument errors
+"""The C-ABI library: it loads without a GPU, exports every symbol the headers in
+include/ declare, its host-side preparation agrees with the oracle, and argument errors
 come back before anything is launched (CPU only; no kernel runs here)."""
 import ctypes
 import os
@@ -23,7 +23,8 @@ def L():
 
 
 def declared_symbols():
-    src = open(os.path.join(ROOT, "include", "rq.h")).read()
+    inc = os.path.join(ROOT, "include")
+    src = "".join(open(os.path.join(inc, f)).read() for f in sorted(os.listdir(inc)) if f.endswith(".h"))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(rq_[a-z0-9_]+)\s*\(", src)))
 
