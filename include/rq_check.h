@@ -32,6 +32,29 @@ extern "C" {
  */
 rq_status rq_convert_check(const float* in, int32_t n, uint8_t* e4m3, uint8_t* e2m1, void* stream);
 
+/*
+ * rq_set_wait_limit -- host.  Every mbarrier wait in the library's kernels is
+ * bounded; this sets the bound, in nanoseconds, for launches made after the
+ * call (from any thread).  0 restores the default of 2 s; values above 20 s
+ * return RQ_ERR_INVALID_ARG.  `previous` (may be NULL) receives the old bound.
+ * A kernel whose wait runs out records a code in the caller's status word
+ * (rq_read_status then returns RQ_ERR_TIMEOUT), stops issuing copies and
+ * MMAs, waits (bounded) for the ones already issued, frees its tensor memory
+ * and exits; the outputs of that call are undefined.
+ */
+rq_status rq_set_wait_limit(uint64_t limit_ns, uint64_t* previous);
+
+/*
+ * rq_set_fault_injection -- host, test hook.  While `extra_tx_bytes` is non-zero,
+ * the first operand load of every CTA of later launches (the first row group of
+ * the activation and weight kernels, the first K stage of the GEMM kernels)
+ * announces that many more bytes than its copies bring.  Every copy still
+ * lands; only the barrier never completes, so the bounded waits on it run out
+ * and the call reports RQ_ERR_TIMEOUT.  0 switches it off.  A multiple of 16,
+ * at most 4096, else RQ_ERR_INVALID_ARG.
+ */
+rq_status rq_set_fault_injection(uint32_t extra_tx_bytes);
+
 #ifdef __cplusplus
 }
 #endif

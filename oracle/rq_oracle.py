@@ -39,7 +39,7 @@ import math
 
 import numpy as np
 
-INT4, LM16, NVFP4, LM4 = 1, 2, 3, 4
+INT4, LM16, NVFP4, LM4, INT4A = 1, 2, 3, 4, 5
 
 MASK64 = (1 << 64) - 1
 F32 = np.float32
@@ -148,6 +148,59 @@ def rotate(x: np.ndarray, sign, perm, block: int) -> np.ndarray:
 def rotation_matrix(K: int, sign, perm, block: int) -> np.ndarray:
     """Dense R (FP64), column k = R e_k; for the orthogonality checks only."""
     return rotate(np.eye(K, dtype=np.float64), sign, perm, block).T
+
+
+# ----------------------------------------------------------------------------
+# TR-DQ: zigzag permutation and double block rotation (section 3.2, Eq. 9)
+# ----------------------------------------------------------------------------
+def zigzag_permutation(channel_mag, block: int) -> np.ndarray:
+    """The zigzag permutation P of TR-DQ section 3.2: channels ranked by
+    activation magnitude, largest first (equal magnitudes: lower channel index
+    first), are dealt to the K/block blocks back and forth -- the first
+    K/block to blocks 0, 1, ..., K/block - 1, the next K/block to blocks
+    K/block - 1, ..., 0, and so on -- and inside a block they keep the order in
+    which they were dealt.  Returns perm with output position i reading channel
+    perm[i] (a permutation matrix, orthogonal as the paper notes).
+
+    Pinned by: tests/test_oracle_trdq.py (a hand-dealt K = 8 example, the
+    bijection, and the rank balance between blocks)."""
+    mag = np.asarray(channel_mag, dtype=np.float64)
+    K = mag.size
+    if block < 1 or K % block:
+        raise ValueError("block must divide K")
+    nblk = K // block
+    order = np.lexsort((np.arange(K), -mag))        # magnitude descending, then index
+    perm = np.empty(K, dtype=np.int32)
+    for t, c in enumerate(order):
+        rnd, i = divmod(t, nblk)
+        blk = i if rnd % 2 == 0 else nblk - 1 - i
+        perm[blk * block + rnd] = c
+    return perm
+
+
+def zigzag_from_calibration(calib_f32: np.ndarray, sign, block: int) -> np.ndarray:
+    """Zigzag permutation from calibration tokens (TR-DQ section 3.2): the
+    channel magnitudes are max over tokens of |(x R1)_j|, R1 the first block
+    rotation (signs, no permutation, block FWHT, FP32 contract)."""
+    K = calib_f32.shape[1]
+    y1 = rotate(np.asarray(calib_f32, dtype=F32), sign, np.arange(K, dtype=np.int32), block)
+    return zigzag_permutation(np.max(np.abs(y1), axis=0), block)
+
+
+def rotate_double(x: np.ndarray, sign, zz_perm, block: int) -> np.ndarray:
+    """TR-DQ Eq. 9, activation side: y = R2 P R1 x with R1 the first block
+    rotation (random signs on the natural channel order, orthonormal FWHT per
+    block), P the zigzag permutation and R2 a second orthonormal FWHT per block.
+    Each rotation follows the FP32 contract of ``rotate`` (reading: the two
+    block rotations are RPBH rotations of their own -- signs only on the first,
+    the zigzag as the permutation of the second).  The weight side folds the
+    same R into W (``rotate_quantize(..., double=...)``).
+
+    Pinned by: tests/test_oracle_trdq.py (equal to the product of the dense
+    matrices; orthogonal; cancels inside the layer in FP64)."""
+    K = x.shape[1]
+    y1 = rotate(x, sign, np.arange(K, dtype=np.int32), block)
+    return rotate(y1, np.ones(K, dtype=np.int8), zz_perm, block)
 
 
 # ----------------------------------------------------------------------------
@@ -423,6 +476,36 @@ def quant_int4(y: np.ndarray, group: int | None = None):
     return q.reshape(rows, K), scale
 
 
+def quant_int4_asym(y: np.ndarray):
+    """Asymmetric per-token INT4 (TR-DQ section 3.1, Eq. 1-3): the range
+    [min, max] of the row is mapped onto 0..15.  Reading of the garbled signs:
+    Eq. 3 gives z = round(min/s), and the code is round(x/s) - z, so that min
+    lands on code 0 (adding z, as Eq. 1 prints it, would put min at 2z).  In
+    FP32: inv = 15/(max - min); z = rne(min * inv); q = clamp(rne(y * inv) - z,
+    0, 15); s = (max - min)/15; dequantized x = s (q + z).  The stored nibble is
+    q - 8 (two's complement, -8..7) and the per-token zero point z + 8, so that
+    x = s (nibble + zero point) and the GEMM reads signed nibbles like the
+    symmetric format.  A constant row (max == min, after rotation only the zero
+    row) gets s = 0, nibble -8, zero point 8.
+    Returns (nibble int8, scale float32, zero_point float32).
+
+    Pinned by: tests/test_oracle_trdq.py (hand-worked rows with ties, the
+    clamp at both ends, the error bound s/2, min and max on codes 0 and 15)."""
+    rows, K = y.shape
+    y = np.asarray(y, dtype=F32)
+    mn = np.min(y, axis=1)
+    mx = np.max(y, axis=1)
+    rng = (mx - mn).astype(F32)
+    ok = rng > 0
+    inv = np.where(ok, F32(15.0) / np.where(ok, rng, F32(1.0)), F32(0.0)).astype(F32)
+    z = np.rint((mn * inv).astype(F32))
+    q = np.clip(np.rint((y * inv[:, None]).astype(F32)) - z[:, None], 0, 15)
+    q = np.where(ok[:, None], q, 0)
+    z = np.where(ok, z, 0)
+    scale = np.where(ok, (rng / F32(15.0)).astype(F32), F32(0.0)).astype(F32)
+    return (q - 8).astype(np.int8), scale, (z + 8).astype(F32)
+
+
 def quant_codebook(y: np.ndarray, block: int, boundaries_f32: np.ndarray):
     """Normalise each row to norm sqrt(K) and encode every coordinate as the
     number of codebook boundaries at or below it (OrbitQuant abstract:
@@ -532,7 +615,7 @@ def int4_from_nibble(n: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------
 def rotate_quantize(x_bf16_f32: np.ndarray, fmt: int, block: int, sign, perm,
                     boundaries_f32=None, U_f32=None, weight_rows: bool = False,
-                    group: int = 128):
+                    group: int = 128, zz_perm=None):
     """Rotate, normalise, quantize and pack rows (activation rows, or weight rows
     for W' = W R^T when ``weight_rows``).
 
@@ -541,18 +624,28 @@ def rotate_quantize(x_bf16_f32: np.ndarray, fmt: int, block: int, sign, perm,
     L = bf16(W U) and quantize the full row (y = x_res W^T + c (W U)^T, DiRotQ
     abstract).
 
+    With ``zz_perm``: the TR-DQ double rotation R2 P R1 (``rotate_double``;
+    ``perm`` is then not used).  ``fmt`` INT4A: asymmetric per-token INT4
+    (``quant_int4_asym``; activations only).
+
     Returns a dict with 'codes' (packed uint8), 'q' (unpacked codes), 'scale',
-    'block_scale' (NVFP4, logical rows x K/16) and 'coef' (BF16 bits of c or L)."""
+    'block_scale' (NVFP4, logical rows x K/16), 'zero_point' (INT4A) and 'coef'
+    (BF16 bits of c or L)."""
     x = np.asarray(x_bf16_f32, dtype=F32)
-    out = {"coef": None, "block_scale": None}
+    out = {"coef": None, "block_scale": None, "zero_point": None}
     if U_f32 is not None:
         cf = project_coefficients(x, U_f32)
         cb = _bf16_bits(cf)
         out["coef"] = cb
         if not weight_rows:
             x = residual(x, _bf16_f32(cb), U_f32)
-    y = rotate(x, sign, perm, block)
-    if fmt == INT4:
+    y = rotate(x, sign, perm, block) if zz_perm is None else rotate_double(x, sign, zz_perm, block)
+    if fmt == INT4A:
+        if weight_rows:
+            raise ValueError("asymmetric INT4 is an activation format")
+        q, s, zp = quant_int4_asym(y)
+        out["q"], out["codes"], out["scale"], out["zero_point"] = q, pack_nibbles(q), s, zp
+    elif fmt == INT4:
         q, s = quant_int4(y, group if weight_rows else None)
         out["q"], out["codes"] = q, pack_nibbles(q)
         # weight-row group scales are stored group-major, [K/group][N]
@@ -579,9 +672,13 @@ def _bf16_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(F32)
 
 
-def dequant_values(q: np.ndarray, fmt: int, block_scale=None, centroids_e4m3=None):
+def dequant_values(q: np.ndarray, fmt: int, block_scale=None, centroids_e4m3=None, zero_point=None):
     """FP64 operand values the GEMM multiplies, before the per-row/per-group
-    scales: INT4 integers, e4m3 centroid values, or e2m1 x e4m3 block scale."""
+    scales: INT4 integers (asymmetric: nibble + per-row zero point), e4m3
+    centroid values, or e2m1 x e4m3 block scale."""
+    if fmt == INT4A:
+        n = int4_from_nibble(q) if q.dtype == np.uint8 else q
+        return n.astype(np.float64) + np.asarray(zero_point, np.float64)[:, None]
     if fmt == INT4:
         return int4_from_nibble(q).astype(np.float64) if q.dtype == np.uint8 else q.astype(np.float64)
     if fmt in (LM16, LM4):
@@ -594,16 +691,17 @@ def dequant_values(q: np.ndarray, fmt: int, block_scale=None, centroids_e4m3=Non
 
 
 def reference_gemm(a_fmt: int, w_fmt: int, qa, sa, qw, sw, a_bs=None, w_bs=None,
-                   a_cent=None, w_cent=None, c_bf16=None, L_bf16=None, group: int = 128):
+                   a_cent=None, w_cent=None, c_bf16=None, L_bf16=None, group: int = 128, a_zp=None):
     """FP64 reference output Y (M x N) over the dequantized values:
 
-    * INT4: Y = s_a[m] sum_g s_w[g, n] (sum_{k in g} qa qw), integer partials exact;
+    * INT4: Y = s_a[m] sum_g s_w[g, n] (sum_{k in g} qa qw), integer partials exact
+      (asymmetric activations: qa = nibble + zero point, still integers);
     * codebook / NVFP4: Y = s_a[m] s_w[n] sum_k a_k w_k with dequantized values;
     * plus sum_j c[m, j] L[n, j] when the low-rank branch is present.
 
     ``qa``/``qw`` are unpacked codes (M x K, N x K); INT4 weight scales are
     [K/group, N] (group-major); other weight scales are per row [N]."""
-    A = dequant_values(qa, a_fmt, a_bs, a_cent)
+    A = dequant_values(qa, a_fmt, a_bs, a_cent, a_zp)
     B = dequant_values(qw, w_fmt, w_bs, w_cent)
     if w_fmt == INT4:
         K = A.shape[1]

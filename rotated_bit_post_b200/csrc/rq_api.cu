@@ -2,6 +2,7 @@
 // checking, host-side table preparation and kernel dispatch.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -9,12 +10,19 @@
 #include <vector>
 
 #include "../../include/rq.h"
+#include "../../include/rq_check.h"
 #include "rq_host.h"
 #include "rq_internal.h"
 
 namespace {
 
 thread_local char g_err[512] = "";
+
+// Bounded-wait limit of the kernels and the fault-injection test hook
+// (include/rq_check.h); read at every launch.
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;   // 2 s: far above any legitimate wait
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+std::atomic<uint32_t> g_inject_tx{0};
 
 rq_status fail(rq_status s, const char* fmt, ...) {
   va_list ap;
@@ -91,6 +99,8 @@ rq_status run_k1(int32_t fmt, bool weight, const uint16_t* X, int32_t rows, int3
   a.bscale = bscale;
   a.status = status;
   a.num_sms = num_sms();
+  a.wait_ns = g_wait_ns.load();
+  a.inject_tx = g_inject_tx.load();
   cudaError_t e = rq::launch_k1(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "rotate/quantize launch failed: %s", cudaGetErrorString(e));
   return ok();
@@ -208,10 +218,27 @@ rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int
   g.out_fp32 = out_fp32 ? 1 : 0;
   g.status = status;
   g.num_sms = num_sms();
+  g.wait_ns = g_wait_ns.load();
+  g.inject_tx = g_inject_tx.load();
   const char* why = nullptr;
   cudaError_t e = rq::launch_gemm(g, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess)
     return fail(RQ_ERR_CUDA, "GEMM launch failed: %s%s%s", cudaGetErrorString(e), why ? " / " : "", why ? why : "");
+  return ok();
+}
+
+rq_status rq_set_wait_limit(uint64_t limit_ns, uint64_t* previous) {
+  if (limit_ns == 0) limit_ns = kDefaultWaitNs;
+  if (limit_ns > 20000000000ull) return fail(RQ_ERR_INVALID_ARG, "wait limit above 20 s");
+  const uint64_t old = g_wait_ns.exchange(limit_ns);
+  if (previous) *previous = old;
+  return ok();
+}
+
+rq_status rq_set_fault_injection(uint32_t extra_tx_bytes) {
+  if (extra_tx_bytes % 16 || extra_tx_bytes > 4096)
+    return fail(RQ_ERR_INVALID_ARG, "extra bytes must be a multiple of 16 and at most 4096");
+  g_inject_tx.store(extra_tx_bytes);
   return ok();
 }
 

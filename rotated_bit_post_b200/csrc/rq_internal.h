@@ -28,6 +28,8 @@ struct K1Launch {
   uint8_t* bscale;
   int32_t* status;
   int num_sms;
+  uint64_t wait_ns;        // bounded-wait limit of every mbarrier wait
+  uint32_t inject_tx;      // test hook: extra expect-tx bytes on the first load (0: off)
 };
 
 cudaError_t launch_k1(const K1Launch& a, cudaStream_t st);
@@ -50,6 +52,8 @@ struct GemmLaunch {
   int out_fp32;
   int32_t* status;
   int num_sms;
+  uint64_t wait_ns;
+  uint32_t inject_tx;
 };
 
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why);

@@ -9,9 +9,10 @@
 //
 // Data flow per CTA (persistent over groups of R rows):
 //   HBM --cp.async.bulk--> smem row buffer (mbarrier)
-//   [projection: c = bf16(x U) from the BF16 rows, each of the R x 32 sums a
-//    sequential FP32 chain over k; the rows are widened to FP32 in place and
-//    x_res = x - c U^T (sequential over j) overwrites them]
+//   [projection: c = bf16(x U) from the BF16 rows, each of the R x 32 sums one
+//    sequential FP32 chain per 128-channel chunk, the chunk sums added in
+//    order; the rows are widened to FP32 in place and x_res = x - c U^T
+//    (sequential over j) overwrites them]
 //   a group of L = b/32 lanes owns one b-wide Hadamard block of one row: lane j
 //   of the group holds the 32 consecutive rotated coordinates 32j .. 32j+31,
 //   gathered from smem through the signed-permutation table; butterfly stages
@@ -66,6 +67,8 @@ struct __align__(16) K1Params {
   int32_t lut_shift, lut_gmin, lut_n;
   uint2 lut[K1_LUT_MAX];
   float rcp_e4m3[128];     // fp32(1 / e4m3 value) for the positive e4m3 codes, 0 for code 0
+  uint64_t wait_ns;        // limit of every bounded wait
+  uint32_t inject_tx;      // test hook: extra expect-tx bytes on the CTA's first row group
 };
 
 
@@ -209,6 +212,10 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     mbar_init(&full[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // the GEMM that consumes these codes may be scheduled now: its CTAs only
+    // take SMs this persistent grid leaves free, and it waits for this grid's
+    // completion before reading anything it writes
+    griddep_launch_dependents();
   }
   __syncthreads();
 
@@ -216,7 +223,9 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     const int r0 = g * R;
     const int nr = min(R, p.rows - r0);
     uint16_t* dst = PROJ ? land : xs + (size_t)buf * R * KS;
-    mbar_expect_tx(&full[buf], (uint32_t)nr * row_bytes);
+    // (the test hook overstates the first group's byte count: every row still
+    // lands, the wait for it runs out)
+    mbar_expect_tx(&full[buf], (uint32_t)nr * row_bytes + (g == (int)blockIdx.x ? p.inject_tx : 0u));
     for (int i = 0; i < nr; ++i) bulk_g2s(dst + (size_t)i * KS, p.x + (size_t)(r0 + i) * K, row_bytes, &full[buf]);
   };
 
@@ -255,10 +264,16 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
     const bool has_next = g + (int)gridDim.x < p.ngroups;
     float* part_ss = part_ss2 + (size_t)(it & 1) * R * nblk;
     uint32_t* amax_bits = amax_bits2 + (size_t)(it & 1) * R * ngrp;
-    mbar_wait(&full[buf], PROJ ? (it & 1) : ((it >> 1) & 1), p.status, ST_TIMEOUT_LOAD, abort_flag);
+    const uint32_t par = PROJ ? (it & 1) : ((it >> 1) & 1);
+    mbar_wait(&full[buf], par, p.status, ST_TIMEOUT_LOAD, abort_flag, p.wait_ns);
     // everyone has finished the previous group past this barrier
     __syncthreads();
-    if (*abort_flag) break;
+    if (*abort_flag) {
+      // the rows of this group were the only copies in flight: let them land
+      // (bounded) before the CTA's shared memory goes away
+      if (threadIdx.x == 0) mbar_drain(&full[buf], par, p.wait_ns);
+      break;
+    }
     if constexpr (!PROJ) {
       // prefetch the next group into the other buffer (last read by the
       // previous group's gather)
@@ -723,6 +738,8 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
   p.scale = a.scale;
   p.bscale = a.bscale;
   p.status = a.status;
+  p.wait_ns = a.wait_ns;
+  p.inject_tx = a.inject_tx;
   p.rows = a.rows;
   p.K = a.K;
   p.r = a.r;

@@ -73,6 +73,8 @@ struct __align__(16) GemmParams {
   int out_fp32;
   int tma_store;           // BF16 output written through shared memory + TMA stores
   int32_t* status;
+  uint64_t wait_ns;        // limit of every bounded wait
+  uint32_t inject_tx;      // test hook: extra expect-tx bytes on the first operand stage
 };
 
 // ------------------------------------------------------------------ helpers
@@ -260,6 +262,101 @@ __device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t ta
   ++*sc;
 }
 
+// (x0, x1) * (y0, y1) on one packed FP32 pair
+__device__ __forceinline__ void mul2_f32(float& x0, float& x1, float y0, float y1) {
+  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 b, {%2, %3};\n\t"
+      "mul.rn.f32x2 a, a, b;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(y0), "f"(y1));
+}
+
+// tcgen05.wait::ld that also names the destination registers of the loads it
+// waits for, so that no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld_wait_regs16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
+}
+
+// y for four consecutive columns: acc * (s_a * s_w), on packed FP32 pairs
+__device__ __forceinline__ void scale4(const uint32_t* a, const float* sw, float sa, float (&y)[4]) {
+  const float4 w4 = *reinterpret_cast<const float4*>(sw);
+  float s0 = sa, s1 = sa, s2 = sa, s3 = sa;
+  mul2_f32(s0, s1, w4.x, w4.y);
+  mul2_f32(s2, s3, w4.z, w4.w);
+  y[0] = __uint_as_float(a[0]);
+  y[1] = __uint_as_float(a[1]);
+  y[2] = __uint_as_float(a[2]);
+  y[3] = __uint_as_float(a[3]);
+  mul2_f32(y[0], y[1], s0, s1);
+  mul2_f32(y[2], y[3], s2, s3);
+}
+
+// Epilogue of the 256 x 512 pair tiles: this warp drains 256 accumulator
+// columns of its 32 token rows.  BF16 output: 16 columns at a time, the TMEM
+// load of the next 16 in flight while these are scaled and written to one of
+// this warp's two 2 KB staging buffers; every 32 columns go out as one TMA
+// store.  FP32 output (used for verification): 32 columns at a time, stored
+// straight to global memory, the same FP32 values.
+__device__ __forceinline__ void epi_half_wide(const GemmParams& p, const CUtensorMap* ymap, uint32_t tacc,
+                                              const float* sw, float sa, int row, int n0, int row0, uint32_t stg,
+                                              uint32_t& stc) {
+  const int lane = threadIdx.x & 31;
+  if (!p.tma_store) {
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+      uint32_t a[32];
+      tmem_ld32(tacc + ch * 32, a);
+      tmem_ld_wait();
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        float y[4];
+        scale4(a + i, sw + ch * 32 + i, sa, y);
+        v[i] = y[0]; v[i + 1] = y[1]; v[i + 2] = y[2]; v[i + 3] = y[3];
+      }
+      if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, n0 + ch * 32, v);
+    }
+    return;
+  }
+  uint32_t acc[2][16];
+  tmem_ld16(tacc, acc[0]);
+#pragma unroll
+  for (int hc = 0; hc < 16; ++hc) {
+    tmem_ld_wait_regs16(acc[hc & 1]);
+    if (hc + 1 < 16) tmem_ld16(tacc + (hc + 1) * 16, acc[(hc + 1) & 1]);
+    const uint32_t buf = stg + (stc & 1u) * 2048u;
+    if ((hc & 1) == 0 && stc >= 2) {   // the store two boxes back must have read this buffer
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {   // 8 columns -> one 16-byte shared store of BF16
+      float y0[4], y1[4];
+      scale4(acc[hc & 1] + 8 * c, sw + hc * 16 + 8 * c, sa, y0);
+      scale4(acc[hc & 1] + 8 * c + 4, sw + hc * 16 + 8 * c + 4, sa, y1);
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(y0[0], y0[1]), h1 = __floats2bfloat162_rn(y0[2], y0[3]);
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(y1[0], y1[1]), h3 = __floats2bfloat162_rn(y1[2], y1[3]);
+      const int cc = 2 * (hc & 1) + c;   // 16-byte column of the 32 x 32 box
+      st_shared_v4(buf + lane * 64 + ((cc ^ ((lane >> 1) & 3)) << 4), *reinterpret_cast<uint32_t*>(&h0),
+                   *reinterpret_cast<uint32_t*>(&h1), *reinterpret_cast<uint32_t*>(&h2),
+                   *reinterpret_cast<uint32_t*>(&h3));
+    }
+    if (hc & 1) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(ymap, buf, n0 + (hc >> 1) * 32, row0);   // rows >= M, columns >= N clipped by the map
+        bulk_commit_group();
+      }
+      ++stc;
+    }
+  }
+}
+
 // ====================================================================== FP8
 // Persistent, warp-specialised.  Shared-memory plan (operand buffers 1024-B aligned):
 //   packed A  [SP][128 x 64 B]   (TMA, 64B swizzle)
@@ -275,11 +372,15 @@ struct Fp8Plan {
   // epilogue (4 warps x 2 x 2 KB); BN = 128: three expanded stages and 32 KB
   // of staging (16 grouped epilogue warps x 2 KB, or 4 warps x 2 x 2 KB).
   // PAIR (a CTA pair sharing 256 x 256 tiles): each CTA holds half of the
-  // tile's weight rows, so four expanded stages fit.
+  // tile's weight rows, so four expanded stages fit.  BN = 512 (CTA pairs
+  // only, 256 x 512 tiles): each CTA holds 256 weight rows per stage, two
+  // 128-row halves of the two 256-wide output halves; two or three expanded
+  // stages.
+  static constexpr bool WIDE = BN == 512;
   static constexpr int BR = PAIR ? BN / 2 : BN;       // weight rows held by this CTA
-  static constexpr int SP = PAIR ? 4 : BN == 256 ? (WBITS == 4 ? 4 : 5) : 4;
-  static constexpr int SE = PAIR ? 4 : BN == 256 ? 2 : 3;
-  static constexpr int STG = BN == 256 ? 16384 : 32768;
+  static constexpr int SP = WIDE ? 3 : PAIR ? 4 : BN == 256 ? (WBITS == 4 ? 4 : 5) : 4;
+  static constexpr int SE = WIDE ? 2 : PAIR ? 4 : BN == 256 ? 2 : 3;
+  static constexpr int STG = WIDE ? 32768 : BN >= 256 ? 16384 : 32768;
   static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-wide K tile
   static constexpr int PA = BM * 64, PB = BR * WROW, EA = BM * 128, EB = BR * 128;
   static constexpr bool LR = BN == 128;
@@ -293,7 +394,7 @@ struct Fp8Plan {
   static constexpr int SCS = BN == 128 ? 12 : 4;               // grouped scale ring depth (BN 128 only)
   static constexpr int OFF_STG = (OFF_SC + (SCS * BN * 4 > 2 * BN * 4 ? SCS * BN * 4 : 2 * BN * 4) + 1023) & ~1023;
   static constexpr int OFF_BAR = OFF_STG + STG;
-  static constexpr int NBAR = 2 * SP + 2 * SE + 6 + 4 + 2 * SCS;
+  static constexpr int NBAR = 2 * SP + 2 * SE + 6 + 4 + 2 * SCS + 1;   // + MMA drain after an abort
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(BYTES <= 232448, "shared memory plan exceeds 227 KB");
 };
@@ -311,15 +412,23 @@ struct Fp8Plan {
 // 384.  Otherwise: accumulators at 0 and BN (double-buffered across tiles),
 // low-rank at 384 when BN == 128.
 template <int BN, bool GROUPED>
-constexpr int fp8_threads() { return GROUPED ? 704 : BN == 256 ? 768 : 512; }
+constexpr int fp8_threads() { return GROUPED ? 704 : BN == 512 ? 640 : BN == 256 ? 768 : 512; }
 
 template <int BN, int WBITS, bool GROUPED, bool PAIR = false>
 __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
-  static_assert(!PAIR || (BN == 256 && !GROUPED), "CTA pairs run the 256-wide codebook tiles only");
+  static_assert(!PAIR || ((BN == 256 || BN == 512) && !GROUPED), "CTA pairs run the codebook tiles only");
+  static_assert(BN != 512 || PAIR, "512-wide tiles run on CTA pairs");
   using P = Fp8Plan<BN, WBITS, PAIR>;
+  // WIDE (256 x 512 pair tiles): two N = 256 pair MMAs per K step share the
+  // expanded activation tile, accumulating into TMEM columns 0-255 and 256-511
+  constexpr bool WIDE = P::WIDE;
+  constexpr int MMA_N = WIDE ? 256 : BN;
   constexpr int NW = fp8_threads<BN, GROUPED>() / 32;
-  constexpr int NEPI = GROUPED ? 16 : 4;         // epilogue warps
-  constexpr int EXP0 = 4 + NEPI;                 // first expansion warp
+  // WIDE: epilogue warps 2-9 (two per TMEM lane quadrant, one per 256-column
+  // half), expansion warps 10-19; otherwise epilogue from warp 4
+  constexpr int EPI0 = (BN == 512) ? 2 : 4;      // first epilogue warp
+  constexpr int NEPI = GROUPED ? 16 : (BN == 512) ? 8 : 4;   // epilogue warps
+  constexpr int EXP0 = EPI0 + NEPI;              // first expansion warp
   constexpr int NXW = GROUPED ? 4 : NW - EXP0;   // expansion warps
   constexpr int NXT = NXW * 32;                  // expansion threads
   constexpr int NPART = 3;                       // GROUPED partial buffers
@@ -339,6 +448,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
   uint64_t* lracc_empty = lrdone + 1;      // epilogue read it (epilogue -> MMA)
   uint64_t* scfull = lracc_empty + 1;      // [SCS] group scales landed (TMA -> epilogue)
   uint64_t* scempty = scfull + P::SCS;     // [SCS] epilogue used them (epilogue -> TMA)
+  uint64_t* mdrain = scempty + P::SCS;     // MMA thread's own commits, drained after an abort
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P::NBAR);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
   float* sc_slots = reinterpret_cast<float*>(smem + P::OFF_SC);
@@ -362,12 +472,15 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     // PAIR: efull / accempty of the even CTA count both CTAs' warps; eempty and
     // accfull take one multicast commit arrival in each CTA
     for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], PAIR ? 2 * NXW : NXW); mbar_init(&eempty[i], 1); }
-    for (int i = 0; i < 3; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], PAIR ? 2 * NEPI : NEPI); }
+    // WIDE: accempty[h] counts the warps draining half h (four per CTA)
+    constexpr int ACC_ARRIVALS = WIDE ? 2 * (NEPI / 2) : PAIR ? 2 * NEPI : NEPI;
+    for (int i = 0; i < 3; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], ACC_ARRIVALS); }
     mbar_init(lrfull, 1);
     mbar_init(lrsmem_empty, 1);
     mbar_init(lrdone, 1);
     mbar_init(lracc_empty, NEPI);
     for (int i = 0; i < P::SCS; ++i) { mbar_init(&scfull[i], 1); mbar_init(&scempty[i], NEPI); }
+    mbar_init(mdrain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm.a);
@@ -389,6 +502,9 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // launched as a programmatic dependent of the activation kernel: the
+  // prologue above overlaps its tail; nothing it writes is read before this
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -396,32 +512,52 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
       uint32_t kc = 0;
       int tc = 0;
       uint32_t sgc = 0;                    // group-scale ring counter (GROUPED)
+      int lr_issued = 0;
       for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep, ++tc) {
         const int m0 = (tile / nN) * TM + (int)crank * BM, n0 = (tile % nN) * BN;
         for (int kt = 0; kt < nk; ++kt, ++kc) {
           if constexpr (GROUPED) {
             // this group's weight scales s_w[kt, n0 .. n0+127] (one contiguous row slice)
             const int ss = sgc % P::SCS;
-            if (sgc >= P::SCS && !mbar_wait(&scempty[ss], ((sgc / P::SCS) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+            if (sgc >= P::SCS && !mbar_wait(&scempty[ss], ((sgc / P::SCS) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
             const uint32_t nbytes = (uint32_t)min(128, p.N - n0) * 4;
             mbar_expect_tx(&scfull[ss], nbytes);
             bulk_g2s(sc_slots + ss * 128, p.w_scale + (size_t)kt * p.N + n0, nbytes, &scfull[ss]);
             ++sgc;
           }
           const int s = kc % P::SP;
-          if (kc >= P::SP && !mbar_wait(&pempty[s], ((kc / P::SP) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
-          mbar_expect_tx(&pfull[s], P::PA + P::PB);
+          if (kc >= P::SP && !mbar_wait(&pempty[s], ((kc / P::SP) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
+          // (the test hook overstates the first stage's byte count: the copies
+          // land, the consumers' bounded waits for the stage run out)
+          mbar_expect_tx(&pfull[s], P::PA + P::PB + (kc == 0 ? p.inject_tx : 0u));
           tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * 64, m0, &pfull[s]);
-          tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0 + (int)crank * P::BR, &pfull[s]);
+          if constexpr (WIDE) {
+            // this CTA's 128 rows of each 256-wide half of the tile's weight rows
+            tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0 + (int)crank * 128, &pfull[s]);
+            tma_load_2d(smem + P::OFF_PB + s * P::PB + 128 * P::WROW, &tm.b, kt * P::WROW,
+                        n0 + 256 + (int)crank * 128, &pfull[s]);
+          } else {
+            tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0 + (int)crank * P::BR, &pfull[s]);
+          }
         }
         // the tile's low-rank operands go after its K tiles, so waiting for the
         // previous tile's low-rank MMA never stalls the K-tile prefetch
         if (lr) {
-          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
           mbar_expect_tx(lrfull, BM * 64 + BN * 64);
           tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
           tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
+          ++lr_issued;
         }
+      }
+      if (*abort_flag) {
+        // after an abort: let the copies already issued land (bounded) before
+        // this CTA's shared memory is released
+        for (uint32_t c = kc > (uint32_t)P::SP ? kc - P::SP : 0; c < kc; ++c)
+          mbar_drain(&pfull[c % P::SP], (c / P::SP) & 1, p.wait_ns);
+        for (uint32_t c = sgc > (uint32_t)P::SCS ? sgc - P::SCS : 0; c < sgc; ++c)
+          mbar_drain(&scfull[c % P::SCS], (c / P::SCS) & 1, p.wait_ns);
+        if (lr_issued > 0) mbar_drain(lrfull, (lr_issued - 1) & 1, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -429,15 +565,15 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     if (lane == 0 && crank == 0) {
       // (PAIR: M = 256, the instruction descriptor's M field is M / 16)
       const uint32_t idesc =
-          GROUPED ? idesc_i8(BN) : PAIR ? (idesc_f8(BN) & ~(0x1Fu << 24)) | (16u << 24) : idesc_f8(BN);
+          GROUPED ? idesc_i8(BN) : PAIR ? (idesc_f8(MMA_N) & ~(0x1Fu << 24)) | (16u << 24) : idesc_f8(BN);
       uint32_t kc = 0, gc = 0;
       int tc = 0;
       bool ok = true;
       // The low-rank MMA of a tile is issued after its K loop, when the epilogue
       // has long finished reading the previous tile's low-rank accumulator.
       auto lowrank = [&](int tcx) -> bool {
-        if (!(mbar_wait(lrfull, tcx & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
-              (tcx == 0 || mbar_wait(lracc_empty, (tcx - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag))))
+        if (!(mbar_wait(lrfull, tcx & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
+              (tcx == 0 || mbar_wait(lracc_empty, (tcx - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns))))
           return false;
         tc_fence_after();
         const uint32_t ca = sbase + P::OFF_C, la = sbase + P::OFF_L;
@@ -449,10 +585,40 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         tc_commit(lrsmem_empty);
         return true;
       };
-      for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
+      if constexpr (WIDE) {
+        // single accumulators (all 512 columns): the first MMA of a tile into
+        // either half waits until the epilogue has drained that half of the
+        // previous tile
+        for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
+          for (int kt = 0; kt < nk; ++kt, ++kc) {
+            const int s = kc % P::SE;
+            ok = mbar_wait(&efull[s], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (kt == 0 && tc > 0) {
+                ok = mbar_wait(&accempty[h], (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
+                if (!ok) break;
+                tc_fence_after();
+              }
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_f8_2(tmem + h * 256, smem_desc(a + kk * 32, 16, 1024, 2),
+                          smem_desc(b + h * 128 * 128 + kk * 32, 16, 1024, 2), idesc, (kt == 0 && kk == 0) ? 0u : 1u);
+            }
+            if (!ok) break;
+            tc_commit2_mc(&eempty[s], 0x3);   // the stage is free in both CTAs
+          }
+          if (!ok) break;
+          tc_commit2_mc(&accfull[0], 0x3);
+        }
+      }
+      for (int tile = tile0; tile < ntiles && ok && !WIDE; tile += tstep, ++tc) {
         const uint32_t ab = tc & 1;
         if (!grouped && tc >= 2) {
-          ok = mbar_wait(&accempty[ab], ((tc >> 1) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag);
+          ok = mbar_wait(&accempty[ab], ((tc >> 1) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
         }
@@ -461,13 +627,13 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           if (grouped) {
             buf = gc % NPART;
             if (gc >= NPART) {
-              ok = mbar_wait(&accempty[buf], ((gc / NPART) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag);
+              ok = mbar_wait(&accempty[buf], ((gc / NPART) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
               if (!ok) break;
               tc_fence_after();
             }
           }
           const int s = kc % P::SE;
-          ok = mbar_wait(&efull[s], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag);
+          ok = mbar_wait(&efull[s], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
@@ -500,12 +666,21 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           tc_commit(&accfull[ab]);
         if (lr && !(ok = lowrank(tc))) break;
       }
+      if (!ok) {
+        // after an abort: wait (bounded) for the MMAs already issued before
+        // TMEM and the operand stages are released
+        if constexpr (PAIR)
+          tc_commit2_mc(mdrain, 0x1);
+        else
+          tc_commit(mdrain);
+        mbar_drain(mdrain, 0, p.wait_ns);
+      }
     }
-  } else if (warp >= 4 && warp < EXP0) {
+  } else if (warp >= EPI0 && warp < EXP0) {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 4;
-    const int q = e & 3;                     // TMEM lane quadrant (warp id % 4)
-    const int tid = threadIdx.x - 128;       // 0 .. 32*NEPI-1
+    const int e = warp - EPI0;
+    const int q = warp & 3;                  // TMEM lane quadrant (warp id % 4)
+    const int tid = threadIdx.x - 32 * EPI0; // 0 .. 32*NEPI-1
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint32_t gc = 0;
     uint32_t stc = 0;   // TMA-store chunks issued by this warp
@@ -527,8 +702,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         for (int g = 0; g < nk; ++g, ++gc) {
           const uint32_t buf = gc % NPART;
           const int ss = gc % P::SCS;
-          ok = mbar_wait(&scfull[ss], (gc / P::SCS) & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
-               mbar_wait(&accfull[buf], (gc / NPART) & 1, p.status, ST_TIMEOUT_MMA, abort_flag);
+          ok = mbar_wait(&scfull[ss], (gc / P::SCS) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
+               mbar_wait(&accfull[buf], (gc / NPART) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           const float* sw = sc_slots + ss * 128 + h * 32;
@@ -555,7 +730,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         if (!ok) break;
         const float sa256 = sa * 0.00390625f;
         if (lr) {
-          ok = mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag);
+          ok = mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -600,13 +775,27 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           }
           ++stc;
         }
+      } else if constexpr (WIDE) {
+        const int h = e >> 2;                  // this warp's 256-column half
+        float* sw = sc_slots + (tc & 1) * BN;
+        load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid, 32 * NEPI);
+        epi_bar_n<32 * NEPI>();
+        ok = mbar_wait(&accfull[0], tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+        epi_half_wide(p, &tm.y, tmem + lane_off + h * 256, sw + h * 256, sa, row, n0 + h * 256, m0 + q * 32, stg,
+                      stc);
+        // this half may take the next tile's first MMA
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(&accempty[h], 0);
       } else {
         const uint32_t ab = tc & 1;
         float* sw = sc_slots + ab * BN;
         load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid);
         epi_bar_n<32 * NEPI>();
-        ok = mbar_wait(&accfull[ab], (tc >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag) &&
-             (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag));
+        ok = mbar_wait(&accfull[ab], (tc >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns) &&
+             (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
@@ -640,8 +829,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
       for (int kt = 0; kt < nk; ++kt, ++kc) {
         const int sp = kc % P::SP, se = kc % P::SE;
-        ok = mbar_wait(&pfull[sp], (kc / P::SP) & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
-             (kc < P::SE || mbar_wait(&eempty[se], ((kc / P::SE) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag));
+        ok = mbar_wait(&pfull[sp], (kc / P::SP) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
+             (kc < P::SE || mbar_wait(&eempty[se], ((kc / P::SE) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns));
         if (!ok) break;
         const uint32_t pa = sbase + P::OFF_PA + sp * P::PA, pb = sbase + P::OFF_PB + sp * P::PB;
         const uint32_t ea = sbase + P::OFF_EA + se * P::EA, eb = sbase + P::OFF_EB + se * P::EB;
@@ -784,7 +973,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
       // the even CTA's last commits land in this CTA's barriers: wait for them
       // before this CTA may leave
       for (uint32_t c = kc > (uint32_t)P::SE ? kc - P::SE : 0; ok && c < kc; ++c)
-        ok = mbar_wait(&eempty[c % P::SE], (c / P::SE) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag);
+        ok = mbar_wait(&eempty[c % P::SE], (c / P::SE) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns);
     }
   }
 
@@ -819,7 +1008,7 @@ struct Nvf4Plan {
   static constexpr int OFF_L = OFF_C + (LR ? BM * 64 : 0);
   static constexpr int OFF_SC = OFF_L + (LR ? BN * 64 : 0);
   static constexpr int OFF_BAR = OFF_SC + 2 * BN * 4;
-  static constexpr int NBAR = 2 * S + 4 + 4 + 8;
+  static constexpr int NBAR = 2 * S + 4 + 4 + 8 + 2;   // + MMA and scale-copy drains after an abort
   static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
   static_assert(BYTES <= 232448, "shared memory plan exceeds 227 KB");
 };
@@ -852,6 +1041,8 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
   uint64_t* lracc_empty = lrdone + 1;
   uint64_t* sffull = lracc_empty + 1;      // [4] scale factors in TMEM (copy warp -> MMA)
   uint64_t* sfempty = sffull + 4;          // [4] MMAs done with a slot (MMA -> copy warp)
+  uint64_t* mdrain = sfempty + 4;          // MMA thread's own commits, drained after an abort
+  uint64_t* cdrain = mdrain + 1;           // scale-copy thread's own commits, likewise
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P::NBAR);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
   float* sc_slots = reinterpret_cast<float*>(smem + P::OFF_SC);
@@ -871,6 +1062,8 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
     mbar_init(lrdone, 1);
     mbar_init(lracc_empty, 8);
     for (int i = 0; i < 4; ++i) { mbar_init(&sffull[i], 1); mbar_init(&sfempty[i], 1); }
+    mbar_init(mdrain, 1);
+    mbar_init(cdrain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm.a);
@@ -884,6 +1077,9 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // launched as a programmatic dependent of the activation kernel: the
+  // prologue above overlaps its tail; nothing it writes is read before this
+  griddep_wait();
   constexpr uint32_t SF_COLS = 16 + 4 * (BN / 32);   // SFA 4 x 4 columns + SFB 4 x BN/32
   constexpr int SF_SLOTS = 4;
 
@@ -891,6 +1087,7 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
     if (lane == 0) {
       uint32_t kc = 0;
       int tc = 0;
+      int lr_issued = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tc) {
         const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
         const uint8_t* sfa_src = p.a_bscale + (size_t)(m0 / 128) * ktiles64 * 512;
@@ -898,9 +1095,9 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
         const int nb_valid = min(BN / 128, (p.N + 127) / 128 - n0 / 128);
         for (int kt = 0; kt < nk; ++kt, ++kc) {
           const int s = kc % P::S;
-          if (kc >= P::S && !mbar_wait(&empty[s], ((kc / P::S) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          if (kc >= P::S && !mbar_wait(&empty[s], ((kc / P::S) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
           uint8_t* st = smem + s * P::STAGE;
-          mbar_expect_tx(&full[s], P::PA + P::PB + P::SA + nb_valid * 2048);
+          mbar_expect_tx(&full[s], P::PA + P::PB + P::SA + nb_valid * 2048 + (kc == 0 ? p.inject_tx : 0u));
           tma_load_2d(st, &tm.a, kt * 128, m0, &full[s]);
           tma_load_2d(st + P::PA, &tm.b, kt * 128, n0, &full[s]);
           // 4 scale chunks (k tiles of 64) x 512 B, contiguous in the K1 layout
@@ -910,11 +1107,17 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
                      p.w_bscale + ((size_t)(n0 / 128 + nb) * ktiles64 + (size_t)kt * 4) * 512, 2048, &full[s]);
         }
         if (lr) {   // after the K tiles (see the codebook kernel)
-          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) break;
+          if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
           mbar_expect_tx(lrfull, BM * 64 + BN * 64);
           tma_load_2d(smem + P::OFF_C, &tm.c, 0, m0, lrfull);
           tma_load_2d(smem + P::OFF_L, &tm.l, 0, n0, lrfull);
+          ++lr_issued;
         }
+      }
+      if (*abort_flag) {   // let the copies already issued land (bounded)
+        for (uint32_t c = kc > (uint32_t)P::S ? kc - P::S : 0; c < kc; ++c)
+          mbar_drain(&full[c % P::S], (c / P::S) & 1, p.wait_ns);
+        if (lr_issued > 0) mbar_drain(lrfull, (lr_issued - 1) & 1, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -926,15 +1129,15 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
         const uint32_t ab = tc % P::NACC;
         if (tc >= P::NACC) {
-          ok = mbar_wait(&accempty[ab], ((tc / P::NACC) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag);
+          ok = mbar_wait(&accempty[ab], ((tc / P::NACC) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
         }
         for (int kt = 0; kt < nk; ++kt, ++kc) {
           const int s = kc % P::S;
           const int sl = kc % SF_SLOTS;
-          ok = mbar_wait(&full[s], (kc / P::S) & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
-               mbar_wait(&sffull[sl], (kc / SF_SLOTS) & 1, p.status, ST_TIMEOUT_FULL, abort_flag);
+          ok = mbar_wait(&full[s], (kc / P::S) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
+               mbar_wait(&sffull[sl], (kc / SF_SLOTS) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = sbase + s * P::STAGE;
@@ -950,8 +1153,8 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
         tc_commit(&accfull[ab]);
         if (lr) {
           // low-rank MMA after the K loop (see the codebook kernel)
-          ok = mbar_wait(lrfull, tc & 1, p.status, ST_TIMEOUT_FULL, abort_flag) &&
-               (tc == 0 || mbar_wait(lracc_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag));
+          ok = mbar_wait(lrfull, tc & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
+               (tc == 0 || mbar_wait(lracc_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns));
           if (!ok) break;
           tc_fence_after();
           const uint32_t ca = sbase + P::OFF_C, la = sbase + P::OFF_L;
@@ -962,6 +1165,10 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
           tc_commit(lrdone);
           tc_commit(lrsmem_empty);
         }
+      }
+      if (!ok) {   // wait (bounded) for the MMAs already issued
+        tc_commit(mdrain);
+        mbar_drain(mdrain, 0, p.wait_ns);
       }
     }
   } else if (warp == 2) {
@@ -976,8 +1183,8 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
           const int s = kc % P::S;
           const int sl = kc % SF_SLOTS;
           ok = (kc < (uint32_t)SF_SLOTS ||
-                mbar_wait(&sfempty[sl], ((kc / SF_SLOTS) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag)) &&
-               mbar_wait(&full[s], (kc / P::S) & 1, p.status, ST_TIMEOUT_FULL, abort_flag);
+                mbar_wait(&sfempty[sl], ((kc / SF_SLOTS) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) &&
+               mbar_wait(&full[s], (kc / P::S) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sfa = sbase + s * P::STAGE + P::PA + P::PB, sfb = sfa + P::SA;
@@ -991,6 +1198,10 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
           }
           tc_commit(&sffull[sl]);
         }
+      }
+      if (!ok) {   // wait (bounded) for the scale copies already issued
+        tc_commit(cdrain);
+        mbar_drain(cdrain, 0, p.wait_ns);
       }
     }
   } else if (warp >= 4) {
@@ -1008,8 +1219,8 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
       float* sw = sc_slots + (tc & 1) * BN;
       load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid, 256);
       epi_bar_n<256>();
-      ok = mbar_wait(&accfull[ab], (tc / P::NACC) & 1, p.status, ST_TIMEOUT_MMA, abort_flag) &&
-           (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag));
+      ok = mbar_wait(&accfull[ab], (tc / P::NACC) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns) &&
+           (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
@@ -1061,12 +1272,24 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Every GEMM launch is a programmatic dependent launch (the kernels call
+// griddep_wait() before touching their inputs), so its prologue overlaps the
+// tail of the previous kernel on the stream, normally the activation kernel.
 template <class Kern>
 cudaError_t launch(Kern k, int smem, dim3 grid, int threads, const TMaps& tm, const GemmParams& gp, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, threads, smem, st>>>(tm, gp);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, tm, gp);
 }
 
 // CTA-pair kernels: clusters of two, as many pairs as can be resident at once
@@ -1076,18 +1299,20 @@ cudaError_t launch_pair(Kern k, int smem, int pairs, int threads, const TMaps& t
                         cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;   // the occupancy query below sees the cluster shape only
   // resident-pair counts per kernel, computed once (guarded: host threads may
   // launch concurrently)
   static std::mutex mu;
@@ -1112,6 +1337,7 @@ cudaError_t launch_pair(Kern k, int smem, int pairs, int threads, const TMaps& t
       }
   }
   cfg.gridDim = dim3(2 * (pairs < resident ? pairs : resident));
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k, tm, gp);
 }
 
@@ -1129,6 +1355,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   memcpy(gp.w_lut, a.w_lut, 16);
   gp.has_lr = a.c != nullptr;
   gp.Y = a.Y; gp.out_fp32 = a.out_fp32; gp.status = a.status;
+  gp.wait_ns = a.wait_ns; gp.inject_tx = a.inject_tx;
   gp.tma_store = 0;
 
   const bool nvf4 = a.a_fmt == RQ_FMT_NVFP4;
@@ -1163,10 +1390,11 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   }
   ok &= make_map_2d(&tm.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, a.K / 2, a.M, a.K / 2, 64, BM,
                     CU_TENSOR_MAP_SWIZZLE_64B);
-  // 256-wide codebook tiles run on CTA pairs (256 x 256 per pair, each CTA
-  // loading and expanding half of the weight rows)
+  // codebook tiles run on CTA pairs, 256 x 512 per pair: each CTA loads and
+  // expands its 128 token rows once per K step for 512 output columns, and
+  // 128 rows of each 256-wide half of the tile's weight rows
   const bool pair = !grouped && BN == 256;
-  const uint32_t brows = pair ? BN / 2 : BN;
+  const uint32_t brows = pair ? 128 : BN;
   if (w2)
     ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 4, a.N, a.K / 4, 32, brows,
                       CU_TENSOR_MAP_SWIZZLE_32B);
@@ -1176,13 +1404,13 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   if (!ok) { *why = "cuTensorMapEncodeTiled failed"; return cudaErrorInvalidValue; }
   if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<128, true>(), tm, gp, st);
   if (pair) {
-    const int ptiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+    const int ptiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + 511) / 512);
     const int pairs = ptiles < sms / 2 ? ptiles : sms / 2;
     if (w2)
-      return launch_pair(gemm_fp8_kernel<256, 2, false, true>, Fp8Plan<256, 2, true>::BYTES, pairs,
-                         fp8_threads<256, false>(), tm, gp, st);
-    return launch_pair(gemm_fp8_kernel<256, 4, false, true>, Fp8Plan<256, 4, true>::BYTES, pairs,
-                       fp8_threads<256, false>(), tm, gp, st);
+      return launch_pair(gemm_fp8_kernel<512, 2, false, true>, Fp8Plan<512, 2, true>::BYTES, pairs,
+                         fp8_threads<512, false>(), tm, gp, st);
+    return launch_pair(gemm_fp8_kernel<512, 4, false, true>, Fp8Plan<512, 4, true>::BYTES, pairs,
+                       fp8_threads<512, false>(), tm, gp, st);
   }
   if (w2) return launch(gemm_fp8_kernel<128, 2, false>, Fp8Plan<128, 2>::BYTES, grid, fp8_threads<128, false>(), tm, gp, st);
   return launch(gemm_fp8_kernel<128, 4, false>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<128, false>(), tm, gp, st);

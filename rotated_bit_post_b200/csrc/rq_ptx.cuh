@@ -1,16 +1,13 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, bulk/TMA copies, tcgen05
 // (TMEM allocation, UMMA issue, commit, loads) and FP8/FP4 conversions.
-// Every wait here is bounded: after RQ_WAIT_NS nanoseconds it records a
-// timeout in the caller's status word and returns false, so no kernel can
-// spin forever on a copy or an MMA that never completes.
+// Every wait here is bounded: after the launch's wait limit (nanoseconds, a
+// kernel parameter; 2 s unless a test lowers it) it records a timeout in the
+// caller's status word and returns false, so no kernel can spin forever on a
+// copy or an MMA that never completes.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
-
-#ifndef RQ_WAIT_NS
-#define RQ_WAIT_NS 2000000000ull  // 2 s: far above any legitimate wait
-#endif
 
 namespace rq {
 
@@ -85,13 +82,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait. Returns false (and records `code` in *status) on timeout or
 // when another thread has already flagged an abort in *abort_flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status, int32_t code,
-                                          volatile int32_t* abort_flag) {
+                                          volatile int32_t* abort_flag, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort_flag && *abort_flag) return false;
-    if (globaltimer() - t0 > RQ_WAIT_NS) {
+    if (globaltimer() - t0 > limit_ns) {
       if (status) atomicCAS(status, 0, code);
       if (abort_flag) *abort_flag = 1;
       return false;
@@ -99,8 +96,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
   }
 }
 
+// Bounded wait used after an abort to let copies or MMAs that were already
+// issued finish before the CTA frees its memory: it ignores the abort flag and
+// records nothing, and gives up after limit_ns.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 <= limit_ns) {
+  }
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialization may start while the previous grid on the stream still runs;
+// griddep_wait() blocks until that grid has completed and its memory writes
+// are visible.  griddep_launch_dependents() lets the next grid be scheduled
+// (it still waits for this one in griddep_wait()).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- bulk copies

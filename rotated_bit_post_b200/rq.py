@@ -39,6 +39,8 @@ SIGNATURES = [
     ("rq_last_error", ctypes.c_char_p, []),
     # include/rq_check.h
     ("rq_convert_check", _c_i32, [_c_p, _c_i32, _c_p, _c_p, _c_p]),
+    ("rq_set_wait_limit", _c_i32, [_c_u64, _c_p]),
+    ("rq_set_fault_injection", _c_i32, [ctypes.c_uint32]),
 ]
 
 
@@ -167,6 +169,19 @@ def rq_convert_check(x, e4m3_out, e2m1_out, stream=None):
     hardware conversions the activation kernel uses (include/rq_check.h)."""
     _check("rq_convert_check", lib().rq_convert_check(_dev(x), x.numel(), _dev(e4m3_out), _dev(e2m1_out),
                                                       _stream(stream)))
+
+
+def rq_set_wait_limit(limit_ns: int) -> int:
+    """Bound of every kernel wait for later launches (0: the 2 s default);
+    returns the previous bound."""
+    prev = ctypes.c_uint64(0)
+    _check("rq_set_wait_limit", lib().rq_set_wait_limit(limit_ns, ctypes.byref(prev)))
+    return prev.value
+
+
+def rq_set_fault_injection(extra_tx_bytes: int):
+    """Test hook: overstate the first operand load's byte count (0: off)."""
+    _check("rq_set_fault_injection", lib().rq_set_fault_injection(extra_tx_bytes))
 
 
 def rq_last_error() -> str:

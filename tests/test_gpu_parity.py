@@ -86,3 +86,11 @@ def test_block_512_and_large_k():
     run_layer(w, 64, 128, check_bf16=False)
     w = dataclasses.replace(inputs.WORKLOADS["c4"], K=16384)
     run_layer(w, 64, 256, check_bf16=False)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,N", [("c3", 640), ("c5", 640), ("c5", 384), ("c4", 384), ("c1", 288), ("c2", 288)])
+def test_ragged_n_after_full_tile(name, N):
+    # a partial output tile after a full one: weight rows past N, their scales
+    # and block scales, and (codebook) a CTA pair whose weight half is empty
+    run_layer(inputs.WORKLOADS[name], 257, N)
