@@ -10,8 +10,10 @@ Weights are folded and quantized once, offline, before timing.
 Prints one JSON line (rank 0).  The headline (top-level ``value``, ``roofline``,
 ``e2e``, ``cpu_baseline``) is the largest single-GPU layer, the Wan-2.1-like
 W2A4 MLP with CFG (65520 tokens x 1536 -> 8960); with ``--config all`` (the
-default) the other four layers are timed in the same run and reported under
-``configs``.  Multi-GPU (torchrun): every rank runs the same layers on its own
+default) the other four layers, and the PixArt-like fc1 layer with the full PCA
+rotation in place of RPBH (``c2p``: K1 is then rq_pca_rotate_quantize_act, a
+BF16 tensor-core product x V plus the split/quantize pass), are timed in the
+same run and reported under ``configs``.  Multi-GPU (torchrun): every rank runs the same layers on its own
 token batches (weak scaling, no collective on the data path); times are the
 max over ranks.  ``--impl reference`` times the CPU oracle on the host cores on
 a bounded sample of the headline workload.  ``--measure-peaks`` times
@@ -38,7 +40,7 @@ from rotated_bit_post_b200 import inputs, multirank  # noqa: E402
 
 METRIC = "W4A4 rotated-linear tokens/s & effective TFLOPS (% FP4/FP8 peak) on 1 B200"
 HEADLINE = "c5"
-ORDER = ["c1", "c2", "c3", "c4", "c5"]
+ORDER = ["c1", "c2", "c3", "c4", "c5", "c2p"]
 L2_FLUSH_BYTES = 256 << 20
 
 # Dense tensor-core work per SM per clock (FLOP), from the instruction rates:
@@ -132,11 +134,30 @@ def flops_per_step(w):
     return 2.0 * w.M * w.N * w.K + 2.0 * w.M * w.N * w.rank
 
 
+def pca_flops(w):
+    """The rotation product y = x V of the full PCA rotation: 2 M K^2."""
+    return 2.0 * w.M * w.K * w.K
+
+
+def pca_rotation_bits(w):
+    """V^T (K x K BF16 bits, row n = eigenvector n): all eigenvectors of the
+    calibration tokens' second moment X^T X / n, dominant first.  A calibrated
+    input of the layer, prepared once on the host like the weights."""
+    cal = inputs.bf16_to_f32(inputs.calibration_tokens(w, n=max(inputs.CALIB_TOKENS, w.K))).astype(np.float64)
+    ev, V = np.linalg.eigh(cal.T @ cal / cal.shape[0])
+    V = V[:, np.argsort(ev)[::-1]]
+    return inputs.bf16_bits(np.ascontiguousarray(V.T).astype(np.float32))
+
+
 def k1_bytes(w):
     """Algorithmic bytes of one activation pass: BF16 read, packed codes, the
-    per-token scale, NVFP4 block scales and the BF16 PCA coefficients."""
+    per-token scale, NVFP4 block scales and the BF16 PCA coefficients (the full
+    PCA rotation adds the FP32 rotated rows, written once and read once, and
+    V once)."""
     from rotated_bit_post_b200 import rq
     per_tok = 2 * w.K + w.K // 2 + 4 + (w.K // 16 if w.a_fmt == rq.NVFP4 else 0) + 2 * w.rank
+    if w.rotation == "pca":
+        return w.M * (per_tok + 8 * w.K) + 2 * w.K * w.K
     return w.M * per_tok
 
 
@@ -210,6 +231,10 @@ class ClockSampler:
 def oracle_step(w, X_bits, W_prep, tables):
     """The oracle's hot path on a sample of rows: rotate/quantize + FP64 GEMM."""
     from oracle import rq_oracle as orc
+    if w.rotation == "pca":
+        oa = orc.quantize_pca(orc.rotate_pca(inputs.bf16_to_f32(X_bits), tables), w.rank)
+        return orc.reference_gemm(orc.INT4, orc.INT4, oa["q"], oa["scale"], W_prep["q"], W_prep["scale"],
+                                  c_bf16=oa["coef"], L_bf16=W_prep["coef"])
     sign, perm, ab, ac, wc, U_f32 = tables
     oa = orc.rotate_quantize(inputs.bf16_to_f32(X_bits), w.a_fmt, w.block, sign, perm, ab, U_f32)
     return orc.reference_gemm(w.a_fmt, w.w_fmt, oa["q"], oa["scale"], W_prep["q"], W_prep["scale"],
@@ -218,6 +243,10 @@ def oracle_step(w, X_bits, W_prep, tables):
 
 def oracle_setup(w):
     from oracle import rq_oracle as orc
+    if w.rotation == "pca":
+        V = inputs.bf16_to_f32(np.ascontiguousarray(pca_rotation_bits(w).T))
+        W_prep = orc.quantize_pca(orc.rotate_pca(inputs.bf16_to_f32(inputs.weights(w)), V), w.rank, weight_rows=True)
+        return W_prep, V
     sign, perm = orc.make_rotation(w.K, w.block, 0)
     ab = ac = wb = wc = None
     if w.a_fmt == orc.LM16:
@@ -360,6 +389,46 @@ class Layer:
         rc, code = self.rq.rq_read_status(self.status)
         if rc != 0:
             raise RuntimeError(f"kernel status {code:#x}")
+
+
+class PcaLayer(Layer):
+    """The same layer with the full PCA rotation: K1 is
+    rq_pca_rotate_quantize_act (y = x V into an FP32 workspace, then the first
+    r coordinates to BF16 and the rest to INT4); K2 is the INT4 GEMM with the
+    rank-r BF16 term, as for the RPBH layer with the projection branch."""
+
+    def __init__(self, w, dev, rank, stream):
+        import torch
+        from rotated_bit_post_b200 import rq
+        self.w, self.dev, self.stream, self.rq = w, dev, stream, rq
+        self.Vt = torch.from_numpy(pca_rotation_bits(w).view(np.int16)).to(dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        Wt = torch.from_numpy(inputs.weights(w).view(np.int16)).to(dev)
+        ws = torch.empty((w.N, w.K), dtype=torch.float32, device=dev)
+        self.wb = {"codes": torch.empty((w.N, w.K // 2), dtype=torch.uint8, device=dev),
+                   "scale": torch.empty((w.K // 128, w.N), dtype=torch.float32, device=dev),
+                   "L": torch.empty((w.N, w.rank), dtype=torch.int16, device=dev), "block_scale": None}
+        rq.rq_pca_quantize_weights(Wt, self.Vt, w.rank, ws, self.wb["L"], self.wb["codes"], self.wb["scale"],
+                                   self.status)
+        del Wt, ws
+        self.X_np = multirank.rank_activations(w, rank)
+        self.X = torch.from_numpy(self.X_np.view(np.int16)).to(dev)
+        self.ab = {"codes": torch.empty((w.M, w.K // 2), dtype=torch.uint8, device=dev),
+                   "scale": torch.empty(w.M, dtype=torch.float32, device=dev),
+                   "c": torch.empty((w.M, w.rank), dtype=torch.int16, device=dev), "block_scale": None}
+        self.ws = torch.empty((w.M, w.K), dtype=torch.float32, device=dev)
+        self.Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+        self.a_bnd = self.a_lut = self.w_lut = None
+        self.check()
+
+    def k1(self, x=None):
+        w, ab = self.w, self.ab
+        self.rq.rq_pca_rotate_quantize_act(self.X if x is None else x, self.Vt, w.rank, self.ws, ab["c"],
+                                           ab["codes"], ab["scale"], self.status, self.stream)
+
+
+def make_layer(w, dev, rank, stream):
+    return (PcaLayer if w.rotation == "pca" else Layer)(w, dev, rank, stream)
 
 
 def time_layer(L, args, flush, dist):
@@ -513,6 +582,17 @@ def layer_result(L, args, t_step, t_k1, t_k2, clocks, dist, world, sms):
                "peak_source": pk["source"] + " copy (MEASURED_PEAKS hbm_gbs)",
                "algorithmic_per_launch": f"{kb} B (2K + K/2 + 4 [+ K/16] [+ 2r] per token)",
                "traffic": None if args.tokens else TRAFFIC["k1"].get(w.name)}
+    if w.rotation == "pca":
+        # the rotation product bounds it: a BF16 contraction of 2 M K^2 FLOP
+        # (the split/quantize pass that follows is in the same time)
+        pf = pca_flops(w)
+        k1_tf = pf / (k1_ms * 1e-3) / 1e12
+        k1_roof = {"kernel": "pca_gemm_kernel + pca_quant_kernel (rq_pca_rotate_quantize_act)", "bound": "tensor",
+                   "achieved": k1_tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": k1_tf / pk["bf16_tflops"],
+                   "peak_source": pk["source"] + " bf16 burst (MEASURED_PEAKS bf16_tflops)",
+                   "algorithmic_per_launch": f"{pf:.4g} FLOP (2MK^2); HBM {kb} B at {k1_gbs:.0f} GB/s "
+                                             f"(2K + 8K + K/2 + 4 + 2r per token, + 2K^2 for V)",
+                   "traffic": None}
     k2_roof = {"kernel": "gemm kernel of rq_w4a4_linear", "bound": "tensor", "achieved": k2_tflops,
                "peak": tp["peak"], "unit": "TFLOP/s", "frac": k2_tflops / tp["peak"],
                "peak_source": tp["peak_source"], "alt_peaks": tp["alt_peaks"],
@@ -546,10 +626,10 @@ def run_ours(args, names, rank, world, dist):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     results = {}
     for name in names:
-        w = inputs.WORKLOADS[name]
+        w = inputs.workload(name)
         if args.tokens:
             w = dataclasses.replace(w, M=args.tokens)
-        L = Layer(w, dev, rank, stream)
+        L = make_layer(w, dev, rank, stream)
         t_step, t_k1, t_k2, clocks = time_layer(L, args, flush, dist)
         res = layer_result(L, args, t_step, t_k1, t_k2, clocks, dist, world, sms)
         if not args.no_bf16_linear:
@@ -564,7 +644,7 @@ def run_ours(args, names, rank, world, dist):
     if rank != 0:
         return
     head = results[HEADLINE] if HEADLINE in results else results[names[-1]]
-    hw = inputs.WORKLOADS[HEADLINE if HEADLINE in results else names[-1]]
+    hw = inputs.workload(HEADLINE if HEADLINE in results else names[-1])
     out = {"metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
            "median_ms_per_step": head["median_ms_per_step"], "higher_is_better": True, "scaling": "weak",
@@ -584,7 +664,7 @@ def run_ours(args, names, rank, world, dist):
         if len(names) > 1:
             for n in names:
                 if n != HEADLINE:
-                    out["configs"][n]["cpu_baseline"] = cpu_baseline(inputs.WORKLOADS[n], 3.0)
+                    out["configs"][n]["cpu_baseline"] = cpu_baseline(inputs.workload(n), 3.0)
             out["configs"][HEADLINE]["cpu_baseline"] = out["cpu_baseline"]
     print(json.dumps(out), flush=True)
 
@@ -656,7 +736,7 @@ def main():
     if args.impl == "reference":
         # the CPU oracle runs once, on rank 0, on the headline layer; other ranks have nothing to do
         if rank == 0:
-            w = inputs.WORKLOADS[HEADLINE if args.config == "all" else args.config]
+            w = inputs.workload(HEADLINE if args.config == "all" else args.config)
             if args.tokens:
                 w = dataclasses.replace(w, M=args.tokens)
             run_reference(args, w, rank, world)

@@ -63,6 +63,10 @@ typedef int32_t rq_status;
 #define RQ_LM16 2  /* 16-level Lloyd-Max codebook index, sign-magnitude nibbles   */
 #define RQ_NVFP4 3 /* E2M1 nibbles + UE4M3 block scale per 16 + FP32 row scale    */
 #define RQ_LM4 4   /* 4-level Lloyd-Max codebook index, 2-bit (weights only)       */
+#define RQ_INT4A 5 /* asymmetric INT4 (activations only): nibble q - 8, per-token
+                      scale s and zero point z + 8, x = s (nibble + zero point)  */
+#define RQ_INT8 6  /* symmetric INT8 (activations only, the W4A8 setting): one
+                      byte per code in -127..127, per-token scale amax/127       */
 
 /*
  * rq_make_rotation -- host.  Draw the RPBH rotation for K channels.
@@ -70,7 +74,7 @@ typedef int32_t rq_status;
  *   rotation"); TR-DQ section 3.2 (a permutation is an orthogonal matrix;
  *   Eq. 8 block-diagonal structure with K / block blocks).
  *   K      number of input channels, K % block == 0.
- *   block  Hadamard block size, a power of two, 128 <= block <= 512 for the
+ *   block  Hadamard block size, a power of two, 16 <= block <= 1024 for the
  *          device calls (any power of two >= 2 here).
  *   seed   64-bit seed of the SplitMix64 stream: K sign draws first (negative
  *          when bit 63 is set), then a Fisher-Yates shuffle of 0..K-1 from the
@@ -84,6 +88,21 @@ typedef int32_t rq_status;
  *   sign[perm[j]] x[perm[j]] over j in the block of i.
  */
 rq_status rq_make_rotation(int32_t K, int32_t block, uint64_t seed, int8_t* sign, int32_t* perm, int32_t* rot);
+
+/*
+ * rq_make_zigzag -- host.  TR-DQ's zigzag permutation (TR-DQ section 3.2, the
+ * paragraph before Eq. 9): channels ranked by magnitude (largest first; equal
+ * magnitudes by channel index) are dealt to the K / block blocks back and
+ * forth -- blocks 0, 1, ..., then ..., 1, 0, and so on -- and keep inside a
+ * block the order in which they arrive.  For the double rotation R2 P R1 the
+ * magnitudes are those of the channels after the first block rotation (for
+ * example the maximum of |(x R1)_j| over calibration tokens).
+ *   channel_mag  [in, host, K] finite, >= 0.   K % block == 0.
+ *   perm   [out, host, K] int32: output position i reads channel perm[i] (may be NULL).
+ *   rot2   [out, host, K] int32: the same as a signed permutation without
+ *          signs, the table rq_rotate_quantize_act2 takes as `rot2` (may be NULL).
+ */
+rq_status rq_make_zigzag(const float* channel_mag, int32_t K, int32_t block, int32_t* perm, int32_t* rot2);
 
 /*
  * rq_make_codebook -- host.  Lloyd-Max quantizer for the marginal of one
@@ -122,7 +141,7 @@ rq_status rq_pca_basis(const uint16_t* calib, int32_t n, int32_t K, int32_t r, u
  * run time; TR-DQ section 3.2: dynamic per-token ranges computed online.)
  *   fmt    RQ_INT4 | RQ_LM16 | RQ_NVFP4.
  *   X      [device, M x K] BF16.     M >= 1.  K % block == 0, K <= 16384,
- *          K % 128 == 0 (INT4 / LM16), K % 256 == 0 (NVFP4).
+ *          K % 128 == 0; with U: block 128, 256 or 512 and, for NVFP4, K % 256 == 0.
  *   rot    [device, K] signed permutation from rq_make_rotation.
  *   boundaries [host, levels-1] FP32 codebook boundaries (RQ_LM16), else NULL.
  *   U, r   [device, K x r] BF16 PCA basis and its rank (r == 32, K <= 3072:
@@ -165,6 +184,83 @@ rq_status rq_quantize_weights(int32_t fmt, const uint16_t* W, int32_t N, int32_t
                               int32_t* status, void* stream);
 
 /*
+ * rq_rotate_quantize_act2 -- device, async.  The activation transform without
+ * the low-rank branch, with two additions (TR-DQ: Time-Rotation Diffusion
+ * Quantization):
+ *   - rot2 (optional, [device, K] signed permutation, from rq_make_zigzag):
+ *     the double block rotation of section 3.2, Eq. 9, y = R2 P R1 x: R1 =
+ *     the random signs of `rot` (its permutation must be the identity) and an
+ *     orthonormal Walsh-Hadamard transform per natural block, P = rot2's
+ *     permutation (its sign bits must be clear), R2 a second per-block
+ *     transform.  Without rot2 the rotation is the one of `rot`, as in
+ *     rq_rotate_quantize_act.
+ *   - fmt RQ_INT8: 8-bit activations for the W4A8 setting (Tables 1-5): inv =
+ *     127 / amax, q = clamp(rne(y inv), -127, 127), one byte per code (codes
+ *     [device, M x K]), scale[m] = amax / 127.
+ *   - fmt RQ_INT4A: asymmetric INT4 (section 3.1, Eq. 1-3, per token): inv =
+ *     15 / (max - min), z = rne(min inv), q = clamp(rne(y inv) - z, 0, 15),
+ *     nibble q - 8; scale[m] = (max - min) / 15 and zero_point[m] = z + 8
+ *     ([device, M] FP32), so that x = scale (nibble + zero point).  A row with
+ *     max == min gets scale 0, nibbles -8 and zero point 8.
+ * Other arguments as rq_rotate_quantize_act; block: any power of two from 16
+ * to 1024 dividing K.  zero_point is required for RQ_INT4A, else ignored.
+ */
+rq_status rq_rotate_quantize_act2(int32_t fmt, const uint16_t* X, int32_t M, int32_t K, int32_t block,
+                                  const int32_t* rot, const int32_t* rot2, const float* boundaries, uint8_t* codes,
+                                  float* scale, float* zero_point, uint8_t* block_scale, int32_t* status,
+                                  void* stream);
+
+/*
+ * rq_quantize_weights2 -- device, async.  Weight preparation without the
+ * low-rank branch, with the optional double rotation `rot2` (as above; the
+ * rows of W are folded with the same R2 P R1) and, for INT4 weights, the
+ * optional output zsum ([device, N] FP32): for each row n, the sum over its
+ * 128-wide groups g, in group order, of scale[g, n] times the sum of the
+ * group's codes.  rq_w4a4_linear2 takes it for the zero-point term of
+ * asymmetric activations.  Other arguments as rq_quantize_weights.
+ */
+rq_status rq_quantize_weights2(int32_t fmt, const uint16_t* W, int32_t N, int32_t K, int32_t block,
+                               const int32_t* rot, const int32_t* rot2, const float* boundaries, uint8_t* codes,
+                               float* scale, uint8_t* block_scale, float* zsum, int32_t* status, void* stream);
+
+/*
+ * rq_pca_rotate_quantize_act -- device, async.  DiRotQ's full PCA rotation
+ * (DiRotQ abstract: activations rotated into a calibrated PCA basis, the
+ * coordinates along the dominant directions kept in BF16, the rest quantized
+ * to 4 bits; the inverse rotation folded into the weights offline):
+ * y = x V on the tensor cores (BF16 operands, FP32 accumulation, order of the
+ * additions not specified), then per row c = bf16(y[0:r]) and the INT4 codes
+ * of y with its first r coordinates set to zero (codes 0 there): inv =
+ * 7 / amax, q = rne(y inv), scale = amax / 7 over coordinates r..K-1.
+ * rq_w4a4_linear(RQ_INT4, RQ_INT4, ..., c, L, r) then gives the layer output.
+ *   X      [device, M x K] BF16.  M >= 0, K % 128 == 0, K <= 16384.
+ *   Vt     [device, K x K] BF16, row n = column n of V (V orthogonal: the
+ *          PCA basis of the calibration tokens, all K eigenvectors, dominant
+ *          first).
+ *   r      0 <= r <= K (the GEMM's low-rank term takes r == 32).
+ *   workspace [device, M x K] FP32, caller-allocated scratch: y is written
+ *          there (and may be read back; it is the rotated activation).
+ *   c_out  [device, M x r] BF16 (may be NULL when r == 0).
+ *   codes  [device, M x K/2] packed nibbles.  scale [device, M] FP32.
+ *   All device pointers 16-byte aligned; status as above.
+ */
+rq_status rq_pca_rotate_quantize_act(const uint16_t* X, int32_t M, int32_t K, const uint16_t* Vt, int32_t r,
+                                     float* workspace, uint16_t* c_out, uint8_t* codes, float* scale,
+                                     int32_t* status, void* stream);
+
+/*
+ * rq_pca_quantize_weights -- device, async.  The weight side of the PCA
+ * rotation: every row w_n becomes w_n V (x W^T = (x V)(W V)^T for orthogonal
+ * V); L = bf16((W V)[:, 0:r]) and the INT4 codes of W V with its first r
+ * coordinates zeroed, one scale per 128 coordinates ([K/128][N] group-major,
+ * the layout rq_w4a4_linear reads).  Arguments as for the activations with
+ * N rows; workspace [device, N x K] FP32.
+ */
+rq_status rq_pca_quantize_weights(const uint16_t* W, int32_t N, int32_t K, const uint16_t* Vt, int32_t r,
+                                  float* workspace, uint16_t* L_out, uint8_t* codes, float* scale,
+                                  int32_t* status, void* stream);
+
+/*
  * rq_w4a4_linear -- device, async.  The 4-bit x 4-bit GEMM on rotated codes with
  * per-token x per-group (INT4) or per-token x per-row scales, plus the optional
  * low-rank term (OrbitQuant abstract: the rotation cancels inside each linear
@@ -175,7 +271,8 @@ rq_status rq_quantize_weights(int32_t fmt, const uint16_t* W, int32_t N, int32_t
  * centroids, or E2M1 x UE4M3 block scale) and one group spanning all of K for
  * non-INT4 weights.
  *   a_fmt/w_fmt  (RQ_INT4, RQ_INT4) | (RQ_LM16, RQ_LM16) | (RQ_LM16, RQ_LM4) |
- *          (RQ_NVFP4, RQ_NVFP4).
+ *          (RQ_NVFP4, RQ_NVFP4) | (RQ_INT8, RQ_INT4): W4A8, 8-bit activation
+ *          codes (from rq_rotate_quantize_act2) against INT4 weights.
  *   a_codes/w_codes, a_scale/w_scale, a_bscale/w_bscale: as produced above.
  *   a_lut/w_lut  [host, 16 / 4 bytes] E4M3 value of each codebook index
  *          (rq_make_codebook's centroids_e4m3) for LM formats; NULL otherwise.
@@ -191,6 +288,19 @@ rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int
                          const float* w_scale, const uint8_t* w_bscale, const uint8_t* a_lut,
                          const uint8_t* w_lut, const uint16_t* c, const uint16_t* L, int32_t r, void* Y,
                          int32_t out_fp32, int32_t* status, void* stream);
+
+/*
+ * rq_w4a4_linear2 -- device, async.  The GEMM for asymmetric INT4 activations
+ * (RQ_INT4A, from rq_rotate_quantize_act2) and INT4 weights (TR-DQ section
+ * 3.1, Eq. 1-3: x = s (nibble + z)):
+ *   Y[m, n] = a_scale[m] * ( sum_g w_scale[g, n] sum_{k in g} a(m, k) w(n, k)
+ *                            + a_zero_point[m] * w_zsum[n] )
+ * with a(m, k) the signed nibbles and w_zsum from rq_quantize_weights2.
+ * Shapes and other arguments as rq_w4a4_linear (no low-rank branch).
+ */
+rq_status rq_w4a4_linear2(int32_t M, int32_t N, int32_t K, const uint8_t* a_codes, const float* a_scale,
+                          const float* a_zero_point, const uint8_t* w_codes, const float* w_scale,
+                          const float* w_zsum, void* Y, int32_t out_fp32, int32_t* status, void* stream);
 
 /*
  * rq_read_status -- synchronises `stream`, reads the device status word and

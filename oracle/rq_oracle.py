@@ -39,7 +39,7 @@ import math
 
 import numpy as np
 
-INT4, LM16, NVFP4, LM4, INT4A = 1, 2, 3, 4, 5
+INT4, LM16, NVFP4, LM4, INT4A, INT8 = 1, 2, 3, 4, 5, 6
 
 MASK64 = (1 << 64) - 1
 F32 = np.float32
@@ -392,6 +392,37 @@ def pca_basis(calib_f32: np.ndarray, r: int):
 PROJ_CHUNK = 128
 
 
+def rotate_pca(x_f32: np.ndarray, V_f32: np.ndarray) -> np.ndarray:
+    """DiRotQ's full rotation (DiRotQ abstract: the activations rotated into a
+    PCA basis, the dominant coordinates kept at higher precision): y = x V with
+    V the K x K basis (BF16 values).  Reading: the plain definition, the sum of
+    the (exact) products formed in FP64 and rounded once to FP32 -- a tensor
+    core's FP32 accumulation is held to it by an error bound, not bit for bit.
+
+    Pinned by: tests/test_oracle_pca_full.py (exact on integer inputs, against
+    a float64 loop, orthogonal V preserves norms)."""
+    return (np.asarray(x_f32, np.float64) @ np.asarray(V_f32, np.float64)).astype(F32)
+
+
+def quantize_pca(y_f32: np.ndarray, r: int, fmt: int = INT4, weight_rows: bool = False, group: int = 128):
+    """The DiRotQ split of a rotated row (DiRotQ abstract): the first r
+    coordinates (the dominant principal directions) kept in BF16 as c, the
+    remaining ones quantized.  Reading: the quantized row keeps all K
+    positions with the first r set to zero (codes 0), so that the 4-bit GEMM
+    runs over K and c L^T adds the r coordinates back.  INT4: per-token absmax
+    (activations) or one scale per 128 coordinates (weight rows).
+    Returns dict(q, codes, scale, coef)."""
+    y = np.asarray(y_f32, F32)
+    coef = _bf16_bits(np.ascontiguousarray(y[:, :r]))
+    ylo = y.copy()
+    ylo[:, :r] = 0
+    if fmt != INT4:
+        raise ValueError("the PCA rotation quantizes to INT4")
+    q, s = quant_int4(ylo, group if weight_rows else None)
+    return {"q": q, "codes": pack_nibbles(q), "scale": np.ascontiguousarray(s.T) if weight_rows else s[:, 0],
+            "coef": coef, "block_scale": None, "zero_point": None}
+
+
 def project_coefficients(x_f32: np.ndarray, U_f32: np.ndarray) -> np.ndarray:
     """c = x U in FP32 (DiRotQ abstract: the coefficients of the activation in
     the PCA subspace), returned as FP32 values before their BF16 rounding.
@@ -504,6 +535,24 @@ def quant_int4_asym(y: np.ndarray):
     z = np.where(ok, z, 0)
     scale = np.where(ok, (rng / F32(15.0)).astype(F32), F32(0.0)).astype(F32)
     return (q - 8).astype(np.int8), scale, (z + 8).astype(F32)
+
+
+def quant_int8(y: np.ndarray):
+    """Symmetric per-token INT8 for the W4A8 setting (TR-DQ section 3.1: b-bit
+    uniform quantization with per-token scales for activations, Tables 1-5: W4A8
+    and W8A8): amax = max|y|; inv = 127/amax; q = clamp(rne(y inv), -127, 127);
+    scale = amax/127.  A zero row gets scale 0 and codes 0.
+    Returns (q int8, scale float32).
+
+    Pinned by: tests/test_oracle_trdq.py (hand cases with ties, the row
+    maximum on 127, the error bound)."""
+    y = np.asarray(y, dtype=F32)
+    amax = np.max(np.abs(y), axis=1)
+    ok = amax > 0
+    inv = np.where(ok, F32(127.0) / np.where(ok, amax, F32(1.0)), F32(0.0)).astype(F32)
+    q = np.clip(np.rint((y * inv[:, None]).astype(F32)), -127, 127).astype(np.int8)
+    scale = np.where(ok, (amax / F32(127.0)).astype(F32), F32(0.0)).astype(F32)
+    return q, scale
 
 
 def quant_codebook(y: np.ndarray, block: int, boundaries_f32: np.ndarray):
@@ -640,7 +689,12 @@ def rotate_quantize(x_bf16_f32: np.ndarray, fmt: int, block: int, sign, perm,
         if not weight_rows:
             x = residual(x, _bf16_f32(cb), U_f32)
     y = rotate(x, sign, perm, block) if zz_perm is None else rotate_double(x, sign, zz_perm, block)
-    if fmt == INT4A:
+    if fmt == INT8:
+        if weight_rows:
+            raise ValueError("INT8 is an activation format here (W4A8)")
+        q, s = quant_int8(y)
+        out["q"], out["codes"], out["scale"] = q, q.view(np.uint8).copy(), s
+    elif fmt == INT4A:
         if weight_rows:
             raise ValueError("asymmetric INT4 is an activation format")
         q, s, zp = quant_int4_asym(y)
@@ -676,6 +730,8 @@ def dequant_values(q: np.ndarray, fmt: int, block_scale=None, centroids_e4m3=Non
     """FP64 operand values the GEMM multiplies, before the per-row/per-group
     scales: INT4 integers (asymmetric: nibble + per-row zero point), e4m3
     centroid values, or e2m1 x e4m3 block scale."""
+    if fmt == INT8:
+        return np.asarray(q).view(np.int8).astype(np.float64)
     if fmt == INT4A:
         n = int4_from_nibble(q) if q.dtype == np.uint8 else q
         return n.astype(np.float64) + np.asarray(zero_point, np.float64)[:, None]

@@ -20,7 +20,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "librq.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["rq_api.cu", "rq_k1.cu", "rq_k2.cu", "rq_host.cpp", "rq_check.cu"]
+SOURCES = ["rq_api.cu", "rq_k1.cu", "rq_k1r.cu", "rq_k2.cu", "rq_pca.cu", "rq_host.cpp", "rq_check.cu"]
 HEADERS = ["rq_ptx.cuh", "rq_internal.h", "rq_host.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -48,16 +48,24 @@ int num_sms() {
 
 rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows, int32_t K, int32_t block,
                           const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r,
-                          const void* coef, const void* codes, const void* scale, const void* bscale) {
-  const bool fmt_ok = fmt == RQ_INT4 || fmt == RQ_LM16 || fmt == RQ_NVFP4 || (weight && fmt == RQ_LM4);
+                          const void* coef, const void* codes, const void* scale, const void* bscale,
+                          const int32_t* rot2 = nullptr, const void* zp = nullptr) {
+  const bool fmt_ok = fmt == RQ_INT4 || fmt == RQ_LM16 || fmt == RQ_NVFP4 || (weight && fmt == RQ_LM4) ||
+                      (!weight && (fmt == RQ_INT4A || fmt == RQ_INT8));
   if (!fmt_ok) return fail(RQ_ERR_INVALID_ARG, "unknown or unsupported format %d", fmt);
   if (rows < 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape rows=%d K=%d", rows, K);
-  if (block != 128 && block != 256 && block != 512)
-    return fail(RQ_ERR_UNSUPPORTED, "block %d: the device path supports 128, 256, 512", block);
+  if (block < 16 || block > 1024 || (block & (block - 1)))
+    return fail(RQ_ERR_UNSUPPORTED, "block %d: a power of two from 16 to 1024", block);
+  if (U && block != 128 && block != 256 && block != 512)
+    return fail(RQ_ERR_UNSUPPORTED, "block %d with the low-rank branch: 128, 256 or 512", block);
   if (K % block) return fail(RQ_ERR_INVALID_ARG, "K=%d is not a multiple of block=%d", K, block);
   if (K > 16384) return fail(RQ_ERR_UNSUPPORTED, "K=%d exceeds 16384", K);
   if (K % 128) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of 128", K);
-  if (fmt == RQ_NVFP4 && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs K %% 256 == 0 (K=%d)", K);
+  if (fmt == RQ_NVFP4 && U && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 with the low-rank branch needs K %% 256 == 0 (K=%d)", K);
+  if (rot2 && U) return fail(RQ_ERR_UNSUPPORTED, "the double rotation runs without the low-rank branch");
+  if (fmt == RQ_INT4A && !zp) return fail(RQ_ERR_INVALID_ARG, "asymmetric INT4 needs a zero-point output");
+  if ((fmt == RQ_INT4A || fmt == RQ_INT8) && U) return fail(RQ_ERR_UNSUPPORTED, "format %d runs without the low-rank branch", fmt);
+  if ((rot2 && !aligned16(rot2)) || (zp && !aligned16(zp))) return fail(RQ_ERR_ALIGNMENT, "rot2 / zero point not 16-byte aligned");
   if (!X || !rot || !codes || !scale) return fail(RQ_ERR_INVALID_ARG, "null input/output pointer");
   if ((fmt == RQ_LM16 || fmt == RQ_LM4) && !boundaries)
     return fail(RQ_ERR_INVALID_ARG, "codebook format needs boundaries");
@@ -75,8 +83,10 @@ rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows,
 
 rq_status run_k1(int32_t fmt, bool weight, const uint16_t* X, int32_t rows, int32_t K, int32_t block,
                  const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r, uint16_t* coef,
-                 uint8_t* codes, float* scale, uint8_t* bscale, int32_t* status, void* stream) {
-  rq_status s = check_rows_call(fmt, weight, X, rows, K, block, rot, boundaries, U, r, coef, codes, scale, bscale);
+                 uint8_t* codes, float* scale, uint8_t* bscale, int32_t* status, void* stream,
+                 const int32_t* rot2 = nullptr, float* zp = nullptr, float* wz = nullptr) {
+  rq_status s =
+      check_rows_call(fmt, weight, X, rows, K, block, rot, boundaries, U, r, coef, codes, scale, bscale, rot2, zp);
   if (s != RQ_OK) return s;
   if (rows == 0) return ok();
   rq::K1Launch a{};
@@ -87,9 +97,16 @@ rq_status run_k1(int32_t fmt, bool weight, const uint16_t* X, int32_t rows, int3
   a.K = K;
   a.block = block;
   a.rot = rot;
+  a.rot2 = rot2;
+  a.zp = zp;
+  a.wz = wz;
   a.inv_sqrt_b = (float)(1.0 / std::sqrt((double)block));
   a.sqrtK = std::sqrt((float)K);
   a.nbnd = fmt == RQ_LM16 ? 15 : fmt == RQ_LM4 ? 3 : 0;
+  if (a.nbnd) {   // the boundaries must ascend
+    for (int i = 1; i < a.nbnd; ++i)
+      if (!(boundaries[i] > boundaries[i - 1])) return fail(RQ_ERR_INVALID_ARG, "codebook boundaries must ascend");
+  }
   a.bnd = boundaries;
   a.U = U;
   a.r = U ? r : 0;
@@ -116,6 +133,15 @@ rq_status rq_make_rotation(int32_t K, int32_t block, uint64_t seed, int8_t* sign
   if (K <= 0 || block < 2 || (block & (block - 1)) || K % block)
     return fail(RQ_ERR_INVALID_ARG, "K=%d must be a positive multiple of a power-of-two block (block=%d)", K, block);
   rq::make_rotation(K, seed, sign, perm, rot);
+  return ok();
+}
+
+rq_status rq_make_zigzag(const float* channel_mag, int32_t K, int32_t block, int32_t* perm, int32_t* rot2) {
+  if (!channel_mag || (!perm && !rot2)) return fail(RQ_ERR_INVALID_ARG, "null pointer");
+  if (K <= 0 || block < 1 || K % block) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of block=%d", K, block);
+  for (int i = 0; i < K; ++i)
+    if (!(channel_mag[i] >= 0.f)) return fail(RQ_ERR_INVALID_ARG, "channel magnitudes must be finite and >= 0");
+  rq::make_zigzag(channel_mag, K, block, perm, rot2);
   return ok();
 }
 
@@ -158,12 +184,97 @@ rq_status rq_quantize_weights(int32_t fmt, const uint16_t* W, int32_t N, int32_t
   return run_k1(fmt, true, W, N, K, block, rot, boundaries, U, r, L_out, codes, scale, block_scale, status, stream);
 }
 
+rq_status rq_rotate_quantize_act2(int32_t fmt, const uint16_t* X, int32_t M, int32_t K, int32_t block,
+                                  const int32_t* rot, const int32_t* rot2, const float* boundaries, uint8_t* codes,
+                                  float* scale, float* zero_point, uint8_t* block_scale, int32_t* status,
+                                  void* stream) {
+  return run_k1(fmt, false, X, M, K, block, rot, boundaries, nullptr, 0, nullptr, codes, scale, block_scale, status,
+                stream, rot2, zero_point, nullptr);
+}
+
+rq_status rq_quantize_weights2(int32_t fmt, const uint16_t* W, int32_t N, int32_t K, int32_t block,
+                               const int32_t* rot, const int32_t* rot2, const float* boundaries, uint8_t* codes,
+                               float* scale, uint8_t* block_scale, float* zsum, int32_t* status, void* stream) {
+  if (zsum && fmt != RQ_INT4) return fail(RQ_ERR_INVALID_ARG, "code sums are an output of INT4 weights");
+  if (zsum && !aligned16(zsum)) return fail(RQ_ERR_ALIGNMENT, "zsum not 16-byte aligned");
+  return run_k1(fmt, true, W, N, K, block, rot, boundaries, nullptr, 0, nullptr, codes, scale, block_scale, status,
+                stream, rot2, nullptr, zsum);
+}
+
+static rq_status pca_impl(bool weight, const uint16_t* X, int32_t rows, int32_t K, const uint16_t* Vt, int32_t r,
+                          float* workspace, uint16_t* coef, uint8_t* codes, float* scale, int32_t* status,
+                          void* stream) {
+  if (rows < 0 || K <= 0 || K % 128 || K > 16384)
+    return fail(RQ_ERR_INVALID_ARG, "bad PCA shape rows=%d K=%d (K %% 128 == 0, K <= 16384)", rows, K);
+  if (r < 0 || r > K) return fail(RQ_ERR_INVALID_ARG, "r=%d outside 0..K", r);
+  if (!X || !Vt || !workspace || !codes || !scale || (r > 0 && !coef))
+    return fail(RQ_ERR_INVALID_ARG, "null input/output pointer");
+  if (!aligned16(X) || !aligned16(Vt) || !aligned16(workspace) || !aligned16(codes) || !aligned16(scale))
+    return fail(RQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+  if (rows == 0) return ok();
+  rq::PcaLaunch a{};
+  a.weight = weight ? 1 : 0;
+  a.x = X;
+  a.vt = Vt;
+  a.rows = rows;
+  a.K = K;
+  a.r = r;
+  a.y = workspace;
+  a.coef = coef;
+  a.codes = codes;
+  a.scale = scale;
+  a.status = status;
+  a.num_sms = num_sms();
+  a.wait_ns = g_wait_ns.load();
+  cudaError_t e = rq::launch_pca(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "PCA rotation launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+rq_status rq_pca_rotate_quantize_act(const uint16_t* X, int32_t M, int32_t K, const uint16_t* Vt, int32_t r,
+                                     float* workspace, uint16_t* c_out, uint8_t* codes, float* scale,
+                                     int32_t* status, void* stream) {
+  return pca_impl(false, X, M, K, Vt, r, workspace, c_out, codes, scale, status, stream);
+}
+
+rq_status rq_pca_quantize_weights(const uint16_t* W, int32_t N, int32_t K, const uint16_t* Vt, int32_t r,
+                                  float* workspace, uint16_t* L_out, uint8_t* codes, float* scale,
+                                  int32_t* status, void* stream) {
+  return pca_impl(true, W, N, K, Vt, r, workspace, L_out, codes, scale, status, stream);
+}
+
+static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int32_t K, const uint8_t* a_codes,
+                             const float* a_scale, const uint8_t* a_bscale, const float* a_zp, const uint8_t* w_codes,
+                             const float* w_scale, const uint8_t* w_bscale, const float* w_zsum,
+                             const uint8_t* a_lut, const uint8_t* w_lut, const uint16_t* c, const uint16_t* L,
+                             int32_t r, void* Y, int32_t out_fp32, int32_t* status, void* stream);
+
 rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int32_t K, const uint8_t* a_codes,
                          const float* a_scale, const uint8_t* a_bscale, const uint8_t* w_codes,
                          const float* w_scale, const uint8_t* w_bscale, const uint8_t* a_lut,
                          const uint8_t* w_lut, const uint16_t* c, const uint16_t* L, int32_t r, void* Y,
                          int32_t out_fp32, int32_t* status, void* stream) {
-  const bool pair_ok = (a_fmt == RQ_INT4 && w_fmt == RQ_INT4) || (a_fmt == RQ_LM16 && w_fmt == RQ_LM16) ||
+  if (a_fmt == RQ_INT4A) return fail(RQ_ERR_UNSUPPORTED, "asymmetric activations go through rq_w4a4_linear2");
+  return linear_impl(a_fmt, w_fmt, M, N, K, a_codes, a_scale, a_bscale, nullptr, w_codes, w_scale, w_bscale, nullptr,
+                     a_lut, w_lut, c, L, r, Y, out_fp32, status, stream);
+}
+
+rq_status rq_w4a4_linear2(int32_t M, int32_t N, int32_t K, const uint8_t* a_codes, const float* a_scale,
+                          const float* a_zero_point, const uint8_t* w_codes, const float* w_scale,
+                          const float* w_zsum, void* Y, int32_t out_fp32, int32_t* status, void* stream) {
+  if (!a_zero_point || !w_zsum) return fail(RQ_ERR_INVALID_ARG, "zero points and weight code sums are required");
+  if (!aligned16(a_zero_point) || !aligned16(w_zsum)) return fail(RQ_ERR_ALIGNMENT, "zero point / code sums not 16-byte aligned");
+  return linear_impl(RQ_INT4A, RQ_INT4, M, N, K, a_codes, a_scale, nullptr, a_zero_point, w_codes, w_scale, nullptr,
+                     w_zsum, nullptr, nullptr, nullptr, nullptr, 0, Y, out_fp32, status, stream);
+}
+
+static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int32_t K, const uint8_t* a_codes,
+                             const float* a_scale, const uint8_t* a_bscale, const float* a_zp, const uint8_t* w_codes,
+                             const float* w_scale, const uint8_t* w_bscale, const float* w_zsum,
+                             const uint8_t* a_lut, const uint8_t* w_lut, const uint16_t* c, const uint16_t* L,
+                             int32_t r, void* Y, int32_t out_fp32, int32_t* status, void* stream) {
+  const bool pair_ok = (a_fmt == RQ_INT4 && w_fmt == RQ_INT4) || (a_fmt == RQ_INT4A && w_fmt == RQ_INT4) ||
+                       (a_fmt == RQ_INT8 && w_fmt == RQ_INT4) || (a_fmt == RQ_LM16 && w_fmt == RQ_LM16) ||
                        (a_fmt == RQ_LM16 && w_fmt == RQ_LM4) || (a_fmt == RQ_NVFP4 && w_fmt == RQ_NVFP4);
   if (!pair_ok) return fail(RQ_ERR_UNSUPPORTED, "format pair (%d, %d) not supported", a_fmt, w_fmt);
   if (M < 0 || N <= 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape M=%d N=%d K=%d", M, N, K);
@@ -191,7 +302,7 @@ rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int
     if (q && !aligned16(q)) return fail(RQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
   if (M == 0) return ok();
   rq::GemmLaunch g{};
-  g.a_fmt = a_fmt;
+  g.a_fmt = a_fmt == RQ_INT4A ? RQ_INT4 : a_fmt;   // the same signed-nibble GEMM, plus the zero-point term
   g.w_fmt = w_fmt;
   g.M = M;
   g.N = N;
@@ -202,7 +313,9 @@ rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int
   g.w_codes = w_codes;
   g.w_scale = w_scale;
   g.w_bscale = w_bscale;
-  if (a_fmt == RQ_INT4) {
+  g.a_zp = a_zp;
+  g.w_zsum = w_zsum;
+  if (a_fmt == RQ_INT4 || a_fmt == RQ_INT4A || a_fmt == RQ_INT8) {
     for (int i = 0; i < 16; ++i) {
       const int v = i < 8 ? i : i - 16;  // two's-complement nibble
       g.a_lut[i] = g.w_lut[i] = rq::e4m3_encode((double)v);

@@ -272,4 +272,26 @@ bool pca_basis(const uint16_t* calib, int n, int K, int r, uint16_t* U, double* 
   return true;
 }
 
+// TR-DQ's zigzag permutation (section 3.2): channels ranked by magnitude,
+// largest first (equal magnitudes: lower index first), dealt to the K/block
+// blocks back and forth (0 .. nblk-1, then nblk-1 .. 0, ...), keeping inside
+// each block the order in which they arrive.  perm[i] is the channel read at
+// position i; rot2 is the same table as a signed permutation (no signs).
+void make_zigzag(const float* mag, int K, int block, int32_t* perm, int32_t* rot2) {
+  std::vector<int> order(K);
+  for (int i = 0; i < K; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return mag[a] > mag[b]; });
+  const int nblk = K / block;
+  std::vector<int32_t> p(K);
+  for (int t = 0; t < K; ++t) {
+    const int rnd = t / nblk, i = t % nblk;
+    const int blk = (rnd % 2 == 0) ? i : nblk - 1 - i;
+    p[(size_t)blk * block + rnd] = order[t];
+  }
+  for (int i = 0; i < K; ++i) {
+    if (perm) perm[i] = p[i];
+    if (rot2) rot2[i] = p[i];
+  }
+}
+
 }  // namespace rq

@@ -8,6 +8,8 @@
 #define RQ_FMT_LM16 2
 #define RQ_FMT_NVFP4 3
 #define RQ_FMT_LM4 4
+#define RQ_FMT_INT4A 5
+#define RQ_FMT_INT8 6
 
 namespace rq {
 
@@ -17,6 +19,7 @@ struct K1Launch {
   const uint16_t* x;
   int rows, K, block;
   const int32_t* rot;
+  const int32_t* rot2;     // double rotation: the second rotation's table, or null
   float inv_sqrt_b, sqrtK;
   int nbnd;
   const float* bnd;        // host, nbnd entries
@@ -25,6 +28,8 @@ struct K1Launch {
   uint16_t* coef;
   uint8_t* codes;
   float* scale;
+  float* zp;               // asymmetric INT4: per-row zero point
+  float* wz;               // INT4 weights: per-row sum over groups of scale x code sum (or null)
   uint8_t* bscale;
   int32_t* status;
   int num_sms;
@@ -33,6 +38,9 @@ struct K1Launch {
 };
 
 cudaError_t launch_k1(const K1Launch& a, cudaStream_t st);
+// the rows-as-lanes activation kernel (every case without the projection)
+bool k1r_supports(const K1Launch& a);
+cudaError_t launch_k1r(const K1Launch& a, cudaStream_t st);
 
 struct GemmLaunch {
   int a_fmt, w_fmt;
@@ -45,6 +53,8 @@ struct GemmLaunch {
   const uint8_t* w_bscale;
   uint8_t a_lut[16];       // e4m3 bytes per code (FP8 path)
   uint8_t w_lut[16];
+  const float* a_zp;       // asymmetric INT4 activations: per-token zero point (or null)
+  const float* w_zsum;     // with a_zp: per weight row, sum_g s_w[g, n] * sum_{k in g} q_w[n, k]
   const uint16_t* c;       // M x r BF16 (low-rank branch) or null
   const uint16_t* L;       // N x r BF16
   int r;
@@ -57,5 +67,23 @@ struct GemmLaunch {
 };
 
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why);
+
+// DiRotQ full PCA rotation: y = x V (FP32, into the caller's workspace), then
+// the first r coordinates to BF16 and the rest to INT4.
+struct PcaLaunch {
+  int weight;              // 1: weight rows (one INT4 scale per 128 coordinates)
+  const uint16_t* x;       // rows x K BF16
+  const uint16_t* vt;      // K x K BF16, row n = column n of V
+  int rows, K, r;
+  float* y;                // rows x K FP32 workspace
+  uint16_t* coef;          // rows x r BF16
+  uint8_t* codes;          // rows x K/2
+  float* scale;            // rows (activations) or K/128 x rows (weights)
+  int32_t* status;
+  int num_sms;
+  uint64_t wait_ns;
+};
+
+cudaError_t launch_pca(const PcaLaunch& a, cudaStream_t st);
 
 }  // namespace rq

@@ -1,4 +1,6 @@
-// K1: fused rotate -> normalise -> quantize -> pack, one pass over each row.
+// K1: fused rotate -> normalise -> quantize -> pack, one pass over each row,
+// for rows with the DiRotQ low-rank projection (the other calls run in
+// rq_k1r.cu unless its shared-memory plan does not fit).
 //
 // Implements the online activation transform of the rotated W4A4 linear layer
 // (OrbitQuant abstract: randomized permuted block-Hadamard (RPBH) rotation,
@@ -796,6 +798,9 @@ cudaError_t launch_k1_ipw(const K1Launch& a, cudaStream_t st) {
   return launch_k1_t<L, FMT, PROJ, WEIGHT, 2>(a, st);
 }
 
+// this kernel serves the calls with the low-rank projection and, for blocks of
+// 128-512, any call whose shared-memory plan the rows-as-lanes kernel
+// (rq_k1r.cu) cannot fit
 template <int L, int FMT>
 cudaError_t launch_k1_mode(const K1Launch& a, cudaStream_t st) {
   const bool proj = a.U != nullptr;
@@ -821,6 +826,20 @@ cudaError_t launch_k1_fmt(const K1Launch& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_k1(const K1Launch& a, cudaStream_t st) {
+  // the rows-as-lanes kernel: for what only it does (double rotation, INT4A,
+  // INT8, the weight code sums, blocks outside 128-512) and where its layout pays: whole rows of 32
+  // tokens per warp (K <= 1536) and enough row groups to fill the GPU twice;
+  // measured on B200: Wan-like K = 1536 169 us against 186 us, while the
+  // PixArt-width, FLUX QKV and FLUX down-projection layers ran faster here
+  const bool only_r = a.rot2 || a.fmt == RQ_FMT_INT4A || a.fmt == RQ_FMT_INT8 || a.wz ||
+                      (a.block != 128 && a.block != 256 && a.block != 512);
+  const int sms = a.num_sms > 0 ? a.num_sms : 148;
+  const bool r_pays = a.K <= 1536 && a.block <= 128 && a.rows >= 32 * 2 * sms;
+  if (k1r_supports(a) && (only_r || (r_pays && !a.U))) {
+    const cudaError_t e = launch_k1r(a, st);
+    if (e != cudaErrorInvalidValue) return e;
+  }
+  if (only_r) return cudaErrorInvalidValue;
   switch (a.block) {
     case 128: return launch_k1_fmt<4>(a, st);
     case 256: return launch_k1_fmt<8>(a, st);

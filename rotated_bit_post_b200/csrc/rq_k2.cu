@@ -75,6 +75,8 @@ struct __align__(16) GemmParams {
   int32_t* status;
   uint64_t wait_ns;        // limit of every bounded wait
   uint32_t inject_tx;      // test hook: extra expect-tx bytes on the first operand stage
+  const float* a_zp;       // asymmetric INT4 activations: per-token zero point, or null
+  const float* w_zsum;     // per weight row: sum_g s_w[g, n] * (sum of the group's codes)
 };
 
 // ------------------------------------------------------------------ helpers
@@ -365,7 +367,7 @@ __device__ __forceinline__ void epi_half_wide(const GemmParams& p, const CUtenso
 //   e4m3 B    [SE][BN x 128 B]
 //   c / L     [128 x 64 B] / [BN x 64 B] (64B swizzle, BN == 128 only)
 //   weight-scale slots [2][BN] FP32, barriers, TMEM address, abort flag
-template <int BN, int WBITS, bool PAIR = false>
+template <int BN, int WBITS, bool PAIR = false, bool A8 = false>
 struct Fp8Plan {
   // BN = 256: two expanded stages (the expansion, not the MMA, sets the pace),
   // a deeper packed ring and 16 KB of output staging for the TMA-store
@@ -382,7 +384,9 @@ struct Fp8Plan {
   static constexpr int SE = WIDE ? 2 : PAIR ? 4 : BN == 256 ? 2 : 3;
   static constexpr int STG = WIDE ? 32768 : BN >= 256 ? 16384 : 32768;
   static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-wide K tile
-  static constexpr int PA = BM * 64, PB = BR * WROW, EA = BM * 128, EB = BR * 128;
+  // A8 (8-bit activations, W4A8): the activation tile arrives as int8 in the
+  // 128-byte-swizzled layout the MMA reads, straight into the packed stage
+  static constexpr int PA = BM * (A8 ? 128 : 64), PB = BR * WROW, EA = A8 ? 0 : BM * 128, EB = BR * 128;
   static constexpr bool LR = BN == 128;
   static constexpr int OFF_PA = 0;
   static constexpr int OFF_PB = OFF_PA + SP * PA;
@@ -414,11 +418,12 @@ struct Fp8Plan {
 template <int BN, bool GROUPED>
 constexpr int fp8_threads() { return GROUPED ? 704 : BN == 512 ? 640 : BN == 256 ? 768 : 512; }
 
-template <int BN, int WBITS, bool GROUPED, bool PAIR = false>
+template <int BN, int WBITS, bool GROUPED, bool PAIR = false, bool A8 = false>
 __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ GemmParams p) {
   static_assert(!PAIR || ((BN == 256 || BN == 512) && !GROUPED), "CTA pairs run the codebook tiles only");
   static_assert(BN != 512 || PAIR, "512-wide tiles run on CTA pairs");
-  using P = Fp8Plan<BN, WBITS, PAIR>;
+  static_assert(!A8 || GROUPED, "8-bit activations run on the grouped INT4-weight kernel");
+  using P = Fp8Plan<BN, WBITS, PAIR, A8>;
   // WIDE (256 x 512 pair tiles): two N = 256 pair MMAs per K step share the
   // expanded activation tile, accumulating into TMEM columns 0-255 and 256-511
   constexpr bool WIDE = P::WIDE;
@@ -468,7 +473,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
   const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < P::SP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], NXW); }
+    // (A8: the MMA thread also releases each stage, after reading its activation tile)
+    for (int i = 0; i < P::SP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], NXW + (A8 ? 1 : 0)); }
     // PAIR: efull / accempty of the even CTA count both CTAs' warps; eempty and
     // accfull take one multicast commit arrival in each CTA
     for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], PAIR ? 2 * NXW : NXW); mbar_init(&eempty[i], 1); }
@@ -530,7 +536,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           // (the test hook overstates the first stage's byte count: the copies
           // land, the consumers' bounded waits for the stage run out)
           mbar_expect_tx(&pfull[s], P::PA + P::PB + (kc == 0 ? p.inject_tx : 0u));
-          tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * 64, m0, &pfull[s]);
+          tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * (A8 ? 128 : 64), m0, &pfull[s]);
           if constexpr (WIDE) {
             // this CTA's 128 rows of each 256-wide half of the tile's weight rows
             tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0 + (int)crank * 128, &pfull[s]);
@@ -634,9 +640,12 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           }
           const int s = kc % P::SE;
           ok = mbar_wait(&efull[s], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
+          if (A8 && ok)   // the activation tile of this stage (landed before the expansion began)
+            ok = mbar_wait(&pfull[kc % P::SP], (kc / P::SP) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
+          const uint32_t a = A8 ? sbase + P::OFF_PA + (kc % P::SP) * P::PA : sbase + P::OFF_EA + s * P::EA;
+          const uint32_t b = sbase + P::OFF_EB + s * P::EB;
           const bool fresh = grouped || kt == 0;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
@@ -654,6 +663,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
             tc_commit2_mc(&eempty[s], 0x3);   // the stage is free in both CTAs
           else
             tc_commit(&eempty[s]);
+          if constexpr (A8) tc_commit(&pempty[kc % P::SP]);
           if (grouped) {
             tc_commit(&accfull[buf]);
             ++gc;
@@ -728,7 +738,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           }
         }
         if (!ok) break;
-        const float sa256 = sa * 0.00390625f;
+        // codes enter the MMA as 16 v (4-bit) or as themselves (8-bit activations)
+        const float sa256 = sa * (A8 ? 0.0625f : 0.00390625f);
         if (lr) {
           ok = mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
           if (!ok) break;
@@ -747,6 +758,15 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) run[i] *= sa256;
+        }
+        if (p.a_zp) {
+          // asymmetric activations: x = s_a (nibble + z), so the layer adds
+          // s_a z sum_g s_w[g, n] sum_k q_w[n, k] (TR-DQ section 3.1, Eq. 1-3)
+          const float szp = row < p.M ? sa * __ldg(p.a_zp + row) : 0.f;
+          const int nb = n0 + h * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (nb + i < p.N) run[i] = fmaf(szp, __ldg(p.w_zsum + nb + i), run[i]);
         }
         if (!p.tma_store) {
           if (row < p.M) store_row32(p.Y, p.out_fp32, p.N, row, n0 + h * 32, run);
@@ -836,16 +856,19 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         const uint32_t ea = sbase + P::OFF_EA + se * P::EA, eb = sbase + P::OFF_EB + se * P::EB;
         if constexpr (GROUPED) {
           // INT4 codes -> int8 16 v: word j of a 16-byte segment becomes
-          // {even codes << 4, odd codes} (same k order for A and B)
+          // {even codes << 4, odd codes} (same k order for A and B; with
+          // 8-bit activations, which arrive in natural k order, the two
+          // halves are interleaved back into natural order)
           // loads in batches of four: the shared-memory accesses are ordered,
           // so batching keeps four in flight at once
-          constexpr int NIT = 1024 / NXT, NB = 4;
+          // (A8: only the weight codes; the activation tile is already the operand)
+          constexpr int NIT = (A8 ? 512 : 1024) / NXT, NB = 4;
 #pragma unroll
           for (int b0 = 0; b0 < NIT; b0 += NB) {
             uint4 vin[NB];
 #pragma unroll
             for (int j = 0; j < NB; ++j) {
-              const int idx0 = (b0 + j) * NXT + t;
+              const int idx0 = (b0 + j) * NXT + t + (A8 ? 512 : 0);
               const bool isb = idx0 >= 512;
               const int idx = isb ? idx0 - 512 : idx0;
               const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
@@ -853,7 +876,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
             }
 #pragma unroll
             for (int j = 0; j < NB; ++j) {
-              const int idx0 = (b0 + j) * NXT + t;
+              const int idx0 = (b0 + j) * NXT + t + (A8 ? 512 : 0);
               const bool isb = idx0 >= 512;
               const int idx = isb ? idx0 - 512 : idx0;
               const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
@@ -862,8 +885,14 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
               uint32_t o[8];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                o[2 * q] = (w[q] << 4) & 0xF0F0F0F0u;
-                o[2 * q + 1] = w[q] & 0xF0F0F0F0u;
+                const uint32_t lo = (w[q] << 4) & 0xF0F0F0F0u, hi = w[q] & 0xF0F0F0F0u;
+                if constexpr (A8) {
+                  o[2 * q] = __byte_perm(lo, hi, 0x5140);
+                  o[2 * q + 1] = __byte_perm(lo, hi, 0x7362);
+                } else {
+                  o[2 * q] = lo;
+                  o[2 * q + 1] = hi;
+                }
               }
               const uint32_t rowb = dst + r * 128;
               st_shared_v4(rowb + (((2 * seg) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
@@ -1356,6 +1385,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   gp.has_lr = a.c != nullptr;
   gp.Y = a.Y; gp.out_fp32 = a.out_fp32; gp.status = a.status;
   gp.wait_ns = a.wait_ns; gp.inject_tx = a.inject_tx;
+  gp.a_zp = a.a_zp; gp.w_zsum = a.w_zsum;
   gp.tma_store = 0;
 
   const bool nvf4 = a.a_fmt == RQ_FMT_NVFP4;
@@ -1388,8 +1418,13 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
                       CU_TENSOR_MAP_SWIZZLE_64B);
     gp.tma_store = 1;
   }
-  ok &= make_map_2d(&tm.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, a.K / 2, a.M, a.K / 2, 64, BM,
-                    CU_TENSOR_MAP_SWIZZLE_64B);
+  const bool a8 = a.a_fmt == RQ_FMT_INT8;
+  if (a8)   // int8 activation codes: 128-byte rows of the K tile, the MMA's own swizzle
+    ok &= make_map_2d(&tm.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, a.K, a.M, a.K, 128, BM,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    ok &= make_map_2d(&tm.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.a_codes, a.K / 2, a.M, a.K / 2, 64, BM,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
   // codebook tiles run on CTA pairs, 256 x 512 per pair: each CTA loads and
   // expands its 128 token rows once per K step for 512 output columns, and
   // 128 rows of each 256-wide half of the tile's weight rows
@@ -1402,6 +1437,9 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     ok &= make_map_2d(&tm.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w_codes, a.K / 2, a.N, a.K / 2, 64, brows,
                       CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) { *why = "cuTensorMapEncodeTiled failed"; return cudaErrorInvalidValue; }
+  if (grouped && a8)
+    return launch(gemm_fp8_kernel<128, 4, true, false, true>, Fp8Plan<128, 4, false, true>::BYTES, grid,
+                  fp8_threads<128, true>(), tm, gp, st);
   if (grouped) return launch(gemm_fp8_kernel<128, 4, true>, Fp8Plan<128, 4>::BYTES, grid, fp8_threads<128, true>(), tm, gp, st);
   if (pair) {
     const int ptiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + 511) / 512);

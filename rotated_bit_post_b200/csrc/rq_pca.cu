@@ -1,0 +1,285 @@
+// DiRotQ's full PCA rotation (DiRotQ abstract: the activations rotated into a
+// calibrated PCA basis, the coordinates of the dominant directions kept in
+// BF16 and the remaining ones quantized to 4 bits, the inverse rotation folded
+// into the weights offline).
+//
+// Two kernels:
+//  * pca_gemm_kernel: Y = X V, a dense K x K contraction on the tensor cores
+//    (tcgen05.mma kind::f16, BF16 operands, FP32 accumulation in TMEM), TMA-fed,
+//    128 x 256 tiles, persistent, double-buffered accumulators; FP32 output to
+//    the caller's workspace.  The order of the FP32 additions inside the tensor
+//    core is not specified, so this product is held to an error bound, not to
+//    bit equality.
+//  * pca_quant_kernel: per row, the first r coordinates rounded to BF16 (the
+//    coefficients c, or L for weight rows), the others quantized to INT4
+//    (symmetric, absmax per token; one scale per 128 coordinates for weight
+//    rows), the first r positions carrying code 0 so that the 4-bit GEMM runs
+//    over all K positions and c L^T adds them back.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "rq_internal.h"
+#include "rq_ptx.cuh"
+
+namespace rq {
+
+namespace {
+
+constexpr int PBM = 128, PBN = 256, PBK = 64;       // tile; PBK BF16 = 128 bytes per row
+constexpr int PSTAGES = 4;
+constexpr int PA_BYTES = PBM * PBK * 2, PB_BYTES = PBN * PBK * 2;
+constexpr int PSTAGE = PA_BYTES + PB_BYTES;
+constexpr int P_OFF_BAR = PSTAGES * PSTAGE;
+constexpr int P_NBAR = 2 * PSTAGES + 5;   // + the MMA drain barrier
+constexpr int P_SMEM = P_OFF_BAR + P_NBAR * 8 + 16 + 1024;
+constexpr int P_THREADS = 256;   // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
+
+struct __align__(64) PcaMaps {
+  CUtensorMap a;   // X: BF16 [rows][K]
+  CUtensorMap b;   // V^T: BF16 [K][K], row n = column n of V
+};
+
+struct PcaParams {
+  int M, N, K;
+  float* Y;        // [M][N] FP32
+  int32_t* status;
+  uint64_t wait_ns;
+};
+
+__host__ __device__ constexpr uint32_t idesc_bf16_pca() {
+  // F32 accumulator, BF16 A and B (K-major), N = 256, M = 128
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PBN >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(P_THREADS, 1) pca_gemm_kernel(const __grid_constant__ PcaMaps tm,
+                                                                const __grid_constant__ PcaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = full + PSTAGES;
+  uint64_t* accfull = empty + PSTAGES;   // [2]
+  uint64_t* accempty = accfull + 2;      // [2]
+  uint64_t* mdrain = accempty + 2;       // MMAs issued before an abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_NBAR);
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = p.K / PBK;
+  const int nN = (p.N + PBN - 1) / PBN, nM = (p.M + PBM - 1) / PBM;
+  const int ntiles = nM * nN;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < PSTAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+    mbar_init(mdrain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm.a);
+    prefetch_tmap(&tm.b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t kc = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+        const int m0 = (tile / nN) * PBM, n0 = (tile % nN) * PBN;
+        for (int kt = 0; kt < nk; ++kt, ++kc) {
+          const int s = kc % PSTAGES;
+          if (kc >= PSTAGES &&
+              !mbar_wait(&empty[s], ((kc / PSTAGES) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns))
+            break;
+          mbar_expect_tx(&full[s], PSTAGE);
+          tma_load_2d(smem + s * PSTAGE, &tm.a, kt * PBK, m0, &full[s]);
+          tma_load_2d(smem + s * PSTAGE + PA_BYTES, &tm.b, kt * PBK, n0, &full[s]);
+        }
+      }
+      if (*abort_flag)   // let the copies already issued land (bounded)
+        for (uint32_t c = kc > (uint32_t)PSTAGES ? kc - PSTAGES : 0; c < kc; ++c)
+          mbar_drain(&full[c % PSTAGES], (c / PSTAGES) & 1, p.wait_ns);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t kc = 0;
+      int tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+        const uint32_t ab = tc & 1;
+        if (tc >= 2) {
+          ok = mbar_wait(&accempty[ab], ((tc >> 1) - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        for (int kt = 0; kt < nk; ++kt, ++kc) {
+          const int s = kc % PSTAGES;
+          ok = mbar_wait(&full[s], (kc / PSTAGES) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a = sbase + s * PSTAGE, b = a + PA_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // K = 16 per instruction: 32 bytes along the swizzled row
+            umma_bf16(tmem + ab * PBN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
+                      idesc_bf16_pca(), (kt > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&accfull[ab]);
+      }
+      if (!ok) {
+        tc_commit(mdrain);
+        mbar_drain(mdrain, 0, p.wait_ns);
+      }
+    }
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    int tc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+      const int m0 = (tile / nN) * PBM, n0 = (tile % nN) * PBN;
+      const int row = m0 + q * 32 + lane;
+      const uint32_t ab = tc & 1;
+      ok = mbar_wait(&accfull[ab], (tc >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 0; ch < PBN / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + ab * PBN + ch * 32, v);
+        tmem_ld_wait();
+        const int n = n0 + ch * 32;
+        if (row < p.M) {
+          float* dst = p.Y + (size_t)row * p.N + n;
+          if (n + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (n + i < p.N) dst[i] = __uint_as_float(v[i]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[ab]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// One CTA per row: the first r coordinates to BF16, the rest to INT4 with
+// per-token absmax (activations) or one scale per 128 coordinates (weights).
+// The arithmetic of the quantizer is the FP32 contract of the activation
+// kernel: inv = 7 / amax, q = rne(y inv), scale = amax / 7.
+template <bool WEIGHT>
+__global__ void __launch_bounds__(128) pca_quant_kernel(const float* __restrict__ Y, int rows, int K, int r,
+                                                        uint16_t* __restrict__ coef, uint8_t* __restrict__ codes,
+                                                        float* __restrict__ scale) {
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  const float* y = Y + (size_t)row * K;
+  for (int j = threadIdx.x; j < r; j += blockDim.x)
+    coef[(size_t)row * r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(y[j]));
+  __shared__ float red[4];
+  float inv_row = 0.f;
+  if constexpr (!WEIGHT) {
+    float m = 0.f;
+    for (int k = r + threadIdx.x; k < K; k += blockDim.x) m = fmaxf(m, fabsf(y[k]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    const float amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    inv_row = amax > 0.f ? __fdiv_rn(7.0f, amax) : 0.f;
+    if (threadIdx.x == 0) scale[row] = amax > 0.f ? __fdiv_rn(amax, 7.0f) : 0.f;
+  }
+  // 8 coordinates per step: four bytes of packed nibbles
+  for (int c8 = threadIdx.x; c8 < K / 8; c8 += blockDim.x) {
+    const int k0 = c8 * 8;
+    float inv = inv_row;
+    if constexpr (WEIGHT) {
+      // this chunk's 128-wide group: its absmax over the coordinates >= r
+      // (every thread of the group's 16 chunks computes it the same way)
+      const int g0 = (k0 / 128) * 128;
+      float m = 0.f;
+      for (int k = g0; k < g0 + 128; ++k)
+        if (k >= r) m = fmaxf(m, fabsf(y[k]));
+      inv = m > 0.f ? __fdiv_rn(7.0f, m) : 0.f;
+      if (k0 == g0) scale[(size_t)(k0 / 128) * rows + row] = m > 0.f ? __fdiv_rn(m, 7.0f) : 0.f;
+    }
+    uint32_t w = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = k0 + e;
+      const float v = k < r ? 0.f : y[k];
+      const uint32_t b = __float_as_uint(__fadd_rn(__fmul_rn(v, inv), 12582912.0f));
+      w |= (b & 0xFu) << (4 * e);
+    }
+    *reinterpret_cast<uint32_t*>(codes + (size_t)row * (K / 2) + k0 / 2) = w;
+  }
+}
+
+typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<EncodeFn>(f);
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {PBK, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_pca(const PcaLaunch& a, cudaStream_t st) {
+  PcaMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  if (!map_bf16(&tm.a, a.x, a.K, a.rows, PBM) || !map_bf16(&tm.b, a.vt, a.K, a.K, PBN)) return cudaErrorInvalidValue;
+  PcaParams p{a.rows, a.K, a.K, a.y, a.status, a.wait_ns};
+  cudaError_t e = cudaFuncSetAttribute(pca_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  if (e != cudaSuccess) return e;
+  const int ntiles = ((a.rows + PBM - 1) / PBM) * ((a.K + PBN - 1) / PBN);
+  const int sms = a.num_sms > 0 ? a.num_sms : 148;
+  pca_gemm_kernel<<<ntiles < sms ? ntiles : sms, P_THREADS, P_SMEM, st>>>(tm, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.weight)
+    pca_quant_kernel<true><<<a.rows, 128, 0, st>>>(a.y, a.rows, a.K, a.r, a.coef, a.codes, a.scale);
+  else
+    pca_quant_kernel<false><<<a.rows, 128, 0, st>>>(a.y, a.rows, a.K, a.r, a.coef, a.codes, a.scale);
+  return cudaGetLastError();
+}
+
+}  // namespace rq

@@ -40,7 +40,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "Workload", "WORKLOADS", "bf16_bits", "bf16_to_f32", "activations", "weights",
+    "Workload", "WORKLOADS", "PCA_WORKLOADS", "workload", "bf16_bits", "bf16_to_f32", "activations", "weights",
     "calibration_tokens",
 ]
 
@@ -60,6 +60,7 @@ class Workload:
     rank: int
     recipe: str
     description: str
+    rotation: str = "rpbh"   # "pca": the full PCA rotation (rank = BF16 coordinates kept)
 
 
 WORKLOADS = {
@@ -74,6 +75,17 @@ WORKLOADS = {
     "c5": Workload("c5", 65520, 1536, 8960, 128, LM16, LM4, 0, "wan_cfg",
                    "Wan-2.1-1.3B-like video MLP with CFG, W2A4"),
 }
+
+# The PixArt-like fc1 layer again, with the full PCA rotation in place of RPBH
+# plus the rank-32 branch: y = x V, the first 32 coordinates in BF16.
+PCA_WORKLOADS = {
+    "c2p": Workload("c2p", 4096, 1152, 4608, 128, INT4, INT4, 32, "pixart",
+                    "PixArt-like MLP fc1, INT4 W4A4 after the full PCA rotation, 32 coordinates in BF16", "pca"),
+}
+
+
+def workload(name: str) -> Workload:
+    return WORKLOADS[name] if name in WORKLOADS else PCA_WORKLOADS[name]
 
 LAYER_SEED = 0
 TOKEN_SEED = 0

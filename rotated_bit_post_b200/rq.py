@@ -13,8 +13,8 @@ import os
 
 import numpy as np
 
-INT4, LM16, NVFP4, LM4 = 1, 2, 3, 4
-FORMATS = {"int4": INT4, "lm16": LM16, "nvfp4": NVFP4, "lm4": LM4}
+INT4, LM16, NVFP4, LM4, INT4A, INT8 = 1, 2, 3, 4, 5, 6
+FORMATS = {"int4": INT4, "lm16": LM16, "nvfp4": NVFP4, "lm4": LM4, "int4a": INT4A, "int8": INT8}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librq.so")
@@ -35,6 +35,14 @@ SIGNATURES = [
     ("rq_w4a4_linear", _c_i32,
      [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
       _c_i32, _c_p, _c_i32, _c_p, _c_p]),
+    ("rq_make_zigzag", _c_i32, [_c_p, _c_i32, _c_i32, _c_p, _c_p]),
+    ("rq_rotate_quantize_act2", _c_i32,
+     [_c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    ("rq_quantize_weights2", _c_i32,
+     [_c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    ("rq_w4a4_linear2", _c_i32, [_c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p]),
+    ("rq_pca_rotate_quantize_act", _c_i32, [_c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    ("rq_pca_quantize_weights", _c_i32, [_c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
     ("rq_read_status", _c_i32, [_c_p, _c_p, _c_p]),
     ("rq_last_error", ctypes.c_char_p, []),
     # include/rq_check.h
@@ -154,6 +162,54 @@ def rq_w4a4_linear(a_fmt, w_fmt, M, N, K, a_codes, a_scale, a_bscale, w_codes, w
         a_fmt, w_fmt, M, N, K, _dev(a_codes), _dev(a_scale), _dev(a_bscale), _dev(w_codes), _dev(w_scale),
         _dev(w_bscale), _np_ptr(al), _np_ptr(wl), _dev(c), _dev(L), r, _dev(Y), int(out_fp32), _dev(status),
         _stream(stream)))
+
+
+def rq_make_zigzag(channel_mag: np.ndarray, block: int):
+    """-> (perm int32[K], rot2 int32[K]) of TR-DQ's zigzag permutation."""
+    mag = np.ascontiguousarray(channel_mag, np.float32)
+    K = mag.size
+    perm = np.empty(K, np.int32)
+    rot2 = np.empty(K, np.int32)
+    _check("rq_make_zigzag", lib().rq_make_zigzag(_np_ptr(mag), K, block, _np_ptr(perm), _np_ptr(rot2)))
+    return perm, rot2
+
+
+def rq_rotate_quantize_act2(fmt, X, block, rot, rot2, boundaries, codes, scale, zero_point, block_scale, status,
+                            stream=None):
+    M, K = X.shape
+    bnd = None if boundaries is None else np.ascontiguousarray(boundaries, np.float32)
+    _check("rq_rotate_quantize_act2", lib().rq_rotate_quantize_act2(
+        fmt, _dev(X), M, K, block, _dev(rot), _dev(rot2), _np_ptr(bnd), _dev(codes), _dev(scale), _dev(zero_point),
+        _dev(block_scale), _dev(status), _stream(stream)))
+
+
+def rq_pca_rotate_quantize_act(X, Vt, r, workspace, c_out, codes, scale, status, stream=None):
+    M, K = X.shape
+    _check("rq_pca_rotate_quantize_act", lib().rq_pca_rotate_quantize_act(
+        _dev(X), M, K, _dev(Vt), r, _dev(workspace), _dev(c_out), _dev(codes), _dev(scale), _dev(status),
+        _stream(stream)))
+
+
+def rq_pca_quantize_weights(W, Vt, r, workspace, L_out, codes, scale, status, stream=None):
+    N, K = W.shape
+    _check("rq_pca_quantize_weights", lib().rq_pca_quantize_weights(
+        _dev(W), N, K, _dev(Vt), r, _dev(workspace), _dev(L_out), _dev(codes), _dev(scale), _dev(status),
+        _stream(stream)))
+
+
+def rq_quantize_weights2(fmt, W, block, rot, rot2, boundaries, codes, scale, block_scale, zsum, status, stream=None):
+    N, K = W.shape
+    bnd = None if boundaries is None else np.ascontiguousarray(boundaries, np.float32)
+    _check("rq_quantize_weights2", lib().rq_quantize_weights2(
+        fmt, _dev(W), N, K, block, _dev(rot), _dev(rot2), _np_ptr(bnd), _dev(codes), _dev(scale),
+        _dev(block_scale), _dev(zsum), _dev(status), _stream(stream)))
+
+
+def rq_w4a4_linear2(M, N, K, a_codes, a_scale, a_zero_point, w_codes, w_scale, w_zsum, Y, out_fp32, status,
+                    stream=None):
+    _check("rq_w4a4_linear2", lib().rq_w4a4_linear2(
+        M, N, K, _dev(a_codes), _dev(a_scale), _dev(a_zero_point), _dev(w_codes), _dev(w_scale), _dev(w_zsum),
+        _dev(Y), int(out_fp32), _dev(status), _stream(stream)))
 
 
 def rq_read_status(status, stream=None):

@@ -132,3 +132,13 @@ def test_codebook_table_must_be_symmetric(L):
                                 None, None, 0, p, 0, None, None)
         assert code == want, rq.rq_last_error()
     assert "symmetric" in rq.rq_last_error()
+
+
+@pytest.mark.parametrize("K,b,seed", [(8, 2, 0), (1536, 128, 1), (3072, 256, 2)])
+def test_zigzag_matches_oracle(L, K, b, seed):
+    rng = np.random.default_rng(seed)
+    mag = rng.lognormal(0, 2, K).astype(np.float32)
+    mag[::7] = mag[0]            # equal magnitudes rank by channel index on both sides
+    perm, rot2 = rq.rq_make_zigzag(mag, b)
+    assert np.array_equal(perm, orc.zigzag_permutation(mag, b))
+    assert np.array_equal(rot2, perm)

@@ -94,3 +94,13 @@ def test_ragged_n_after_full_tile(name, N):
     # a partial output tile after a full one: weight rows past N, their scales
     # and block scales, and (codebook) a CTA pair whose weight half is empty
     run_layer(inputs.WORKLOADS[name], 257, N)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,block", [("c1", 16), ("c1", 32), ("c1", 64), ("c3", 64), ("c4", 1024),
+                                        ("c3", 1024), ("c5", 512)])
+def test_other_block_sizes(name, block):
+    # power-of-two Hadamard blocks from 16 to 1024 (TR-DQ section 3.2, Eq. 8:
+    # K / 2^n blocks); blocks above 128 span several threads of the kernel
+    w = dataclasses.replace(inputs.WORKLOADS[name], block=block)
+    run_layer(w, 97, 256)

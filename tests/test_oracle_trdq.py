@@ -96,3 +96,23 @@ def test_asym_gemm_is_the_dequantized_product():
     A = s[:, None].astype(np.float64) * (nib + zp[:, None])
     B = qw.astype(np.float64) * np.repeat(sw.T.astype(np.float64), 128, axis=1)
     assert np.allclose(Y, A @ B.T, rtol=1e-12)
+
+
+def test_int8_hand_cases_and_bound():
+    # amax 127 -> inv 1 exactly: ties at .5 go to even, the maximum lands on 127
+    y = np.array([[127.0, 0.5, -0.5, 1.5, -2.5, 126.5, -126.5, 3.0]], dtype=F32)
+    q, s = orc.quant_int8(y)
+    assert list(q[0]) == [127, 0, 0, 2, -2, 126, -126, 3] and s[0] == F32(1.0)
+    q, s = orc.quant_int8(np.zeros((1, 8), F32))
+    assert s[0] == 0 and not q.any()
+    rng = np.random.default_rng(9)
+    y = (rng.standard_normal((30, 256)) * rng.uniform(0.1, 10, (30, 1))).astype(F32)
+    q, s = orc.quant_int8(y)
+    assert np.all(np.abs(q * s[:, None].astype(np.float64) - y) <= s[:, None] * 0.5 * (1 + 1e-6))
+    assert np.all(np.max(np.abs(q.astype(int)), axis=1) == 127)
+    # W4A8: the reference GEMM multiplies the integer codes with the grouped weights
+    qw = rng.integers(-7, 8, (5, 256)).astype(np.int8)
+    sw = rng.uniform(0.1, 1, (2, 5)).astype(F32)
+    Y = orc.reference_gemm(orc.INT8, orc.INT4, q, s, qw, sw)
+    B = qw.astype(np.float64) * np.repeat(sw.T.astype(np.float64), 128, axis=1)
+    assert np.allclose(Y, (q * s[:, None].astype(np.float64)) @ B.T, rtol=1e-12)
