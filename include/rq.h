@@ -261,6 +261,39 @@ rq_status rq_pca_quantize_weights(const uint16_t* W, int32_t N, int32_t K, const
                                   int32_t* status, void* stream);
 
 /*
+ * rq_pca_rotate_quantize_act_noalloc -- device, async.  The paper has no
+ * counterpart: this is rq_pca_rotate_quantize_act for callers that cannot
+ * allocate device memory.  Such callers are, for example, extensions loaded
+ * into a host framework that has reserved the GPU's memory through its own
+ * caching allocator and passes them no allocator (a cudaMalloc there fails
+ * once the pool holds the memory, or forces the framework to give back its
+ * cache), and services that fix their memory budget at start-up and may not
+ * allocate while serving.  They still pass every input and output buffer;
+ * only the FP32 workspace is replaced.
+ *
+ * The workspace is a static device array of RQ_NOALLOC_MAX_ELEMS FP32 values
+ * (16 MiB) inside the library: every GPU that loads the library holds it
+ * until the process exits.  The first call on each device looks up the
+ * array's device address on that device (cudaGetSymbolAddress) and keeps it;
+ * make that first call before any stream capture.  The call allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *
+ *   M * K must not exceed RQ_NOALLOC_MAX_ELEMS; a larger call returns
+ *   RQ_ERR_INVALID_ARG and launches nothing.
+ *   All calls share the one array, which keeps the last call's contents.
+ *   Nothing in it needs to start at zero: the rotation writes every element
+ *   that the split then reads.  Calls that overlap on the GPU (two streams,
+ *   or two host threads, with no ordering between the calls) race on the
+ *   array and give wrong results; order them on one stream.
+ * Other arguments, results and errors as rq_pca_rotate_quantize_act, which
+ * runs the same kernels.
+ */
+#define RQ_NOALLOC_MAX_ELEMS 4194304
+rq_status rq_pca_rotate_quantize_act_noalloc(const uint16_t* X, int32_t M, int32_t K, const uint16_t* Vt, int32_t r,
+                                             uint16_t* c_out, uint8_t* codes, float* scale, int32_t* status,
+                                             void* stream);
+
+/*
  * rq_w4a4_linear -- device, async.  The 4-bit x 4-bit GEMM on rotated codes with
  * per-token x per-group (INT4) or per-token x per-row scales, plus the optional
  * low-rank term (OrbitQuant abstract: the rotation cancels inside each linear

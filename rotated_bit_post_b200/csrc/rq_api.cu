@@ -7,12 +7,20 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "../../include/rq.h"
 #include "../../include/rq_check.h"
 #include "rq_host.h"
 #include "rq_internal.h"
+
+// The workspace of rq_pca_rotate_quantize_act_noalloc: a static device array
+// (one per GPU that loads the library, held until the process exits).  In
+// host code `g_noalloc_scratch` names the host-side stand-in of the symbol,
+// not a device address: the address is looked up once per device, on first
+// use, with that device current (noalloc_scratch below).
+static __device__ __align__(256) float g_noalloc_scratch[RQ_NOALLOC_MAX_ELEMS];
 
 namespace {
 
@@ -121,6 +129,28 @@ rq_status run_k1(int32_t fmt, bool weight, const uint16_t* X, int32_t rows, int3
   cudaError_t e = rq::launch_k1(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "rotate/quantize launch failed: %s", cudaGetErrorString(e));
   return ok();
+}
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_noalloc_once[kMaxDevices];
+float* g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+
+rq_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "cudaGetDevice failed: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(RQ_ERR_UNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = g_noalloc_err[dev] == cudaSuccess ? static_cast<float*>(p) : nullptr;
+  });
+  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev])
+    return fail(RQ_ERR_CUDA, "workspace address lookup failed on device %d: %s", dev,
+                cudaGetErrorString(g_noalloc_err[dev]));
+  *out = g_noalloc_ptr[dev];
+  return RQ_OK;
 }
 
 }  // namespace
@@ -241,6 +271,18 @@ rq_status rq_pca_quantize_weights(const uint16_t* W, int32_t N, int32_t K, const
                                   float* workspace, uint16_t* L_out, uint8_t* codes, float* scale,
                                   int32_t* status, void* stream) {
   return pca_impl(true, W, N, K, Vt, r, workspace, L_out, codes, scale, status, stream);
+}
+
+rq_status rq_pca_rotate_quantize_act_noalloc(const uint16_t* X, int32_t M, int32_t K, const uint16_t* Vt, int32_t r,
+                                             uint16_t* c_out, uint8_t* codes, float* scale, int32_t* status,
+                                             void* stream) {
+  if (M < 0 || K <= 0 || (int64_t)M * K > RQ_NOALLOC_MAX_ELEMS)
+    return fail(RQ_ERR_INVALID_ARG, "M x K = %lld exceeds the built-in workspace of %d FP32 values",
+                (long long)M * K, RQ_NOALLOC_MAX_ELEMS);
+  float* ws = nullptr;
+  const rq_status s = noalloc_scratch(&ws);
+  if (s != RQ_OK) return s;
+  return pca_impl(false, X, M, K, Vt, r, ws, c_out, codes, scale, status, stream);
 }
 
 static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int32_t K, const uint8_t* a_codes,

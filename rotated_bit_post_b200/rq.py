@@ -14,6 +14,7 @@ import os
 import numpy as np
 
 INT4, LM16, NVFP4, LM4, INT4A, INT8 = 1, 2, 3, 4, 5, 6
+NOALLOC_MAX_ELEMS = 4194304   # RQ_NOALLOC_MAX_ELEMS: the built-in workspace of the no-allocation call
 FORMATS = {"int4": INT4, "lm16": LM16, "nvfp4": NVFP4, "lm4": LM4, "int4a": INT4A, "int8": INT8}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -43,6 +44,7 @@ SIGNATURES = [
     ("rq_w4a4_linear2", _c_i32, [_c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p]),
     ("rq_pca_rotate_quantize_act", _c_i32, [_c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
     ("rq_pca_quantize_weights", _c_i32, [_c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    ("rq_pca_rotate_quantize_act_noalloc", _c_i32, [_c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p]),
     ("rq_read_status", _c_i32, [_c_p, _c_p, _c_p]),
     ("rq_last_error", ctypes.c_char_p, []),
     # include/rq_check.h
@@ -188,6 +190,14 @@ def rq_pca_rotate_quantize_act(X, Vt, r, workspace, c_out, codes, scale, status,
     _check("rq_pca_rotate_quantize_act", lib().rq_pca_rotate_quantize_act(
         _dev(X), M, K, _dev(Vt), r, _dev(workspace), _dev(c_out), _dev(codes), _dev(scale), _dev(status),
         _stream(stream)))
+
+
+def rq_pca_rotate_quantize_act_noalloc(X, Vt, r, c_out, codes, scale, status, stream=None):
+    """rq_pca_rotate_quantize_act with the library's built-in workspace (no
+    device allocation; M x K <= NOALLOC_MAX_ELEMS)."""
+    M, K = X.shape
+    _check("rq_pca_rotate_quantize_act_noalloc", lib().rq_pca_rotate_quantize_act_noalloc(
+        _dev(X), M, K, _dev(Vt), r, _dev(c_out), _dev(codes), _dev(scale), _dev(status), _stream(stream)))
 
 
 def rq_pca_quantize_weights(W, Vt, r, workspace, L_out, codes, scale, status, stream=None):
