@@ -65,8 +65,9 @@ typedef int32_t rq_status;
 #define RQ_LM4 4   /* 4-level Lloyd-Max codebook index, 2-bit (weights only)       */
 #define RQ_INT4A 5 /* asymmetric INT4 (activations only): nibble q - 8, per-token
                       scale s and zero point z + 8, x = s (nibble + zero point)  */
-#define RQ_INT8 6  /* symmetric INT8 (activations only, the W4A8 setting): one
-                      byte per code in -127..127, per-token scale amax/127       */
+#define RQ_INT8 6  /* symmetric INT8 (W4A8 / W8A8 settings): one byte per code in
+                      -127..127, scale amax/127 per token (activations) or per
+                      output channel (weight rows)                              */
 
 /*
  * rq_make_rotation -- host.  Draw the RPBH rotation for K channels.
@@ -217,7 +218,10 @@ rq_status rq_rotate_quantize_act2(int32_t fmt, const uint16_t* X, int32_t M, int
  * optional output zsum ([device, N] FP32): for each row n, the sum over its
  * 128-wide groups g, in group order, of scale[g, n] times the sum of the
  * group's codes.  rq_w4a4_linear2 takes it for the zero-point term of
- * asymmetric activations.  Other arguments as rq_quantize_weights.
+ * asymmetric activations.  fmt RQ_INT8: 8-bit weights for the W8A8 setting
+ * (TR-DQ: per-channel weight quantization), the per-token INT8 quantizer
+ * applied to each rotated weight row (codes [device, N x K], scale [device,
+ * N] = amax / 127).  Other arguments as rq_quantize_weights.
  */
 rq_status rq_quantize_weights2(int32_t fmt, const uint16_t* W, int32_t N, int32_t K, int32_t block,
                                const int32_t* rot, const int32_t* rot2, const float* boundaries, uint8_t* codes,
@@ -305,7 +309,11 @@ rq_status rq_pca_rotate_quantize_act_noalloc(const uint16_t* X, int32_t M, int32
  * non-INT4 weights.
  *   a_fmt/w_fmt  (RQ_INT4, RQ_INT4) | (RQ_LM16, RQ_LM16) | (RQ_LM16, RQ_LM4) |
  *          (RQ_NVFP4, RQ_NVFP4) | (RQ_INT8, RQ_INT4): W4A8, 8-bit activation
- *          codes (from rq_rotate_quantize_act2) against INT4 weights.
+ *          codes (from rq_rotate_quantize_act2) against INT4 weights |
+ *          (RQ_INT8, RQ_INT8): W8A8, Y[m, n] = a_scale[m] w_scale[n] sum_k
+ *          q_a q_w (exact integer sums), against weights from
+ *          rq_quantize_weights2.  The 8-bit pairs run without the low-rank
+ *          branch.
  *   a_codes/w_codes, a_scale/w_scale, a_bscale/w_bscale: as produced above.
  *   a_lut/w_lut  [host, 16 / 4 bytes] E4M3 value of each codebook index
  *          (rq_make_codebook's centroids_e4m3) for LM formats; NULL otherwise.

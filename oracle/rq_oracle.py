@@ -690,8 +690,9 @@ def rotate_quantize(x_bf16_f32: np.ndarray, fmt: int, block: int, sign, perm,
             x = residual(x, _bf16_f32(cb), U_f32)
     y = rotate(x, sign, perm, block) if zz_perm is None else rotate_double(x, sign, zz_perm, block)
     if fmt == INT8:
-        if weight_rows:
-            raise ValueError("INT8 is an activation format here (W4A8)")
+        # per token for activations; for weight rows one scale per output
+        # channel (TR-DQ section 3.1, after Eq. 3: per-token activations,
+        # per-channel weights) -- the same per-row quantizer
         q, s = quant_int8(y)
         out["q"], out["codes"], out["scale"] = q, q.view(np.uint8).copy(), s
     elif fmt == INT4A:

@@ -58,8 +58,8 @@ rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows,
                           const int32_t* rot, const float* boundaries, const uint16_t* U, int32_t r,
                           const void* coef, const void* codes, const void* scale, const void* bscale,
                           const int32_t* rot2 = nullptr, const void* zp = nullptr) {
-  const bool fmt_ok = fmt == RQ_INT4 || fmt == RQ_LM16 || fmt == RQ_NVFP4 || (weight && fmt == RQ_LM4) ||
-                      (!weight && (fmt == RQ_INT4A || fmt == RQ_INT8));
+  const bool fmt_ok = fmt == RQ_INT4 || fmt == RQ_LM16 || fmt == RQ_NVFP4 || fmt == RQ_INT8 ||
+                      (weight && fmt == RQ_LM4) || (!weight && fmt == RQ_INT4A);
   if (!fmt_ok) return fail(RQ_ERR_INVALID_ARG, "unknown or unsupported format %d", fmt);
   if (rows < 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape rows=%d K=%d", rows, K);
   if (block < 16 || block > 1024 || (block & (block - 1)))
@@ -99,7 +99,8 @@ rq_status run_k1(int32_t fmt, bool weight, const uint16_t* X, int32_t rows, int3
   if (rows == 0) return ok();
   rq::K1Launch a{};
   a.fmt = fmt;
-  a.weight = weight ? 1 : 0;
+  // INT8 weight rows (per output channel) take the per-token quantizer as is
+  a.weight = weight && fmt != RQ_INT8 ? 1 : 0;
   a.x = X;
   a.rows = rows;
   a.K = K;
@@ -316,7 +317,8 @@ static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N,
                              const uint8_t* a_lut, const uint8_t* w_lut, const uint16_t* c, const uint16_t* L,
                              int32_t r, void* Y, int32_t out_fp32, int32_t* status, void* stream) {
   const bool pair_ok = (a_fmt == RQ_INT4 && w_fmt == RQ_INT4) || (a_fmt == RQ_INT4A && w_fmt == RQ_INT4) ||
-                       (a_fmt == RQ_INT8 && w_fmt == RQ_INT4) || (a_fmt == RQ_LM16 && w_fmt == RQ_LM16) ||
+                       (a_fmt == RQ_INT8 && w_fmt == RQ_INT4) || (a_fmt == RQ_INT8 && w_fmt == RQ_INT8) ||
+                       (a_fmt == RQ_LM16 && w_fmt == RQ_LM16) ||
                        (a_fmt == RQ_LM16 && w_fmt == RQ_LM4) || (a_fmt == RQ_NVFP4 && w_fmt == RQ_NVFP4);
   if (!pair_ok) return fail(RQ_ERR_UNSUPPORTED, "format pair (%d, %d) not supported", a_fmt, w_fmt);
   if (M < 0 || N <= 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape M=%d N=%d K=%d", M, N, K);
@@ -339,6 +341,8 @@ static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N,
   if (w_fmt == RQ_LM16 && !symmetric16(w_lut))
     return fail(RQ_ERR_UNSUPPORTED, "16-level weight table is not symmetric (entry 7-m must be -(entry 8+m))");
   if (c && r != 32) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r == 32 (got %d)", r);
+  if (c && (a_fmt == RQ_INT8 || a_fmt == RQ_INT4A))
+    return fail(RQ_ERR_UNSUPPORTED, "the low-rank branch runs with 4-bit activations");
   const void* ptrs[] = {a_codes, a_scale, w_codes, w_scale, Y, a_bscale, w_bscale, c, L};
   for (const void* q : ptrs)
     if (q && !aligned16(q)) return fail(RQ_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
@@ -376,7 +380,8 @@ static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N,
   g.wait_ns = g_wait_ns.load();
   g.inject_tx = g_inject_tx.load();
   const char* why = nullptr;
-  cudaError_t e = rq::launch_gemm(g, static_cast<cudaStream_t>(stream), &why);
+  cudaError_t e = a_fmt == RQ_INT8 && w_fmt == RQ_INT8 ? rq::launch_gemm_w8a8(g, static_cast<cudaStream_t>(stream))
+                                                       : rq::launch_gemm(g, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess)
     return fail(RQ_ERR_CUDA, "GEMM launch failed: %s%s%s", cudaGetErrorString(e), why ? " / " : "", why ? why : "");
   return ok();

@@ -67,6 +67,8 @@ struct GemmLaunch {
 };
 
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why);
+// W8A8: 8-bit per-token activations x 8-bit per-channel weights (no expansion)
+cudaError_t launch_gemm_w8a8(const GemmLaunch& a, cudaStream_t st);
 
 // DiRotQ full PCA rotation: y = x V (FP32, into the caller's workspace), then
 // the first r coordinates to BF16 and the rest to INT4.

@@ -4,12 +4,16 @@
 // into the weights offline).
 //
 // Two kernels:
-//  * pca_gemm_kernel: Y = X V, a dense K x K contraction on the tensor cores
-//    (tcgen05.mma kind::f16, BF16 operands, FP32 accumulation in TMEM), TMA-fed,
-//    128 x 256 tiles, persistent, double-buffered accumulators; FP32 output to
-//    the caller's workspace.  The order of the FP32 additions inside the tensor
-//    core is not specified, so this product is held to an error bound, not to
-//    bit equality.
+//  * dense_gemm_kernel<false>: Y = X V, a dense K x K contraction on the
+//    tensor cores (tcgen05.mma kind::f16, BF16 operands, FP32 accumulation in
+//    TMEM), TMA-fed, 128 x 256 tiles, persistent, double-buffered
+//    accumulators; FP32 output to the caller's workspace.  The order of the
+//    FP32 additions inside the tensor core is not specified, so this product
+//    is held to an error bound, not to bit equality.
+//    dense_gemm_kernel<true> is the same pipeline on 8-bit operands
+//    (kind::i8, exact S32 accumulation) with a scaled epilogue: the W8A8 GEMM
+//    (TR-DQ, Tables 1-5: 8-bit per-token activations against 8-bit
+//    per-channel weights), Y = s_a[m] s_w[n] sum_k q_a q_w.
 //  * pca_quant_kernel: per row, the first r coordinates rounded to BF16 (the
 //    coefficients c, or L for weight rows), the others quantized to INT4
 //    (symmetric, absmax per token; one scale per 128 coordinates for weight
@@ -29,34 +33,42 @@ namespace rq {
 
 namespace {
 
-constexpr int PBM = 128, PBN = 256, PBK = 64;       // tile; PBK BF16 = 128 bytes per row
+constexpr int PBM = 128, PBN = 256, PROW = 128;     // tile; 128 bytes of K per row per stage
 constexpr int PSTAGES = 4;
-constexpr int PA_BYTES = PBM * PBK * 2, PB_BYTES = PBN * PBK * 2;
+constexpr int PA_BYTES = PBM * PROW, PB_BYTES = PBN * PROW;
 constexpr int PSTAGE = PA_BYTES + PB_BYTES;
 constexpr int P_OFF_BAR = PSTAGES * PSTAGE;
 constexpr int P_NBAR = 2 * PSTAGES + 5;   // + the MMA drain barrier
 constexpr int P_SMEM = P_OFF_BAR + P_NBAR * 8 + 16 + 1024;
 constexpr int P_THREADS = 256;   // warp 0 TMA, warp 1 MMA, warps 4-7 epilogue
 
-struct __align__(64) PcaMaps {
-  CUtensorMap a;   // X: BF16 [rows][K]
-  CUtensorMap b;   // V^T: BF16 [K][K], row n = column n of V
+struct __align__(64) DenseMaps {
+  CUtensorMap a;   // [M][K] K-major: X (BF16) or the activation codes (int8)
+  CUtensorMap b;   // [N][K] K-major: V^T (BF16, row n = column n of V) or the weight codes (int8)
 };
 
-struct PcaParams {
-  int M, N, K;
-  float* Y;        // [M][N] FP32
+struct DenseParams {
+  int M, N, K;         // K in elements
+  void* Y;             // [M][N]: FP32 (BF16 operands), FP32 or BF16 (8-bit operands)
+  int out_fp32;
+  const float* sa;     // 8-bit operands: per-row scales of A [M] and of B [N]
+  const float* sw;
   int32_t* status;
   uint64_t wait_ns;
 };
 
-__host__ __device__ constexpr uint32_t idesc_bf16_pca() {
-  // F32 accumulator, BF16 A and B (K-major), N = 256, M = 128
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PBN >> 3) << 17) | ((uint32_t)(PBM >> 4) << 24);
+// K-major A and B, N = 256, M = 128; BF16 operands with an F32 accumulator,
+// or signed 8-bit operands with an S32 accumulator
+template <bool S8>
+__host__ __device__ constexpr uint32_t idesc_dense() {
+  return (S8 ? (2u << 4) : (1u << 4)) | (1u << 7) | (1u << 10) | ((uint32_t)(PBN >> 3) << 17) |
+         ((uint32_t)(PBM >> 4) << 24);
 }
 
-__global__ void __launch_bounds__(P_THREADS, 1) pca_gemm_kernel(const __grid_constant__ PcaMaps tm,
-                                                                const __grid_constant__ PcaParams p) {
+template <bool S8>
+__global__ void __launch_bounds__(P_THREADS, 1) dense_gemm_kernel(const __grid_constant__ DenseMaps tm,
+                                                                  const __grid_constant__ DenseParams p) {
+  constexpr int PBK = S8 ? 128 : 64;   // elements of K per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -129,9 +141,14 @@ __global__ void __launch_bounds__(P_THREADS, 1) pca_gemm_kernel(const __grid_con
           tc_fence_after();
           const uint32_t a = sbase + s * PSTAGE, b = a + PA_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // K = 16 per instruction: 32 bytes along the swizzled row
-            umma_bf16(tmem + ab * PBN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
-                      idesc_bf16_pca(), (kt > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {   // 32 bytes of K per instruction along the swizzled row
+            if constexpr (S8)
+              umma_i8(tmem + ab * PBN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
+                      idesc_dense<true>(), (kt > 0 || kk > 0) ? 1u : 0u);
+            else
+              umma_bf16(tmem + ab * PBN, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
+                        idesc_dense<false>(), (kt > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit(&empty[s]);
         }
         if (!ok) break;
@@ -154,14 +171,36 @@ __global__ void __launch_bounds__(P_THREADS, 1) pca_gemm_kernel(const __grid_con
       ok = mbar_wait(&accfull[ab], (tc >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
+      const float sa = S8 && row < p.M ? p.sa[row] : 0.f;
 #pragma unroll 1
       for (int ch = 0; ch < PBN / 32; ++ch) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + ab * PBN + ch * 32, v);
         tmem_ld_wait();
         const int n = n0 + ch * 32;
-        if (row < p.M) {
-          float* dst = p.Y + (size_t)row * p.N + n;
+        if constexpr (S8) {
+          if (row < p.M && n < p.N) {   // N % 32 == 0: the chunk is whole
+            float y[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__fmul_rn((float)(int32_t)v[i], sa), __ldg(p.sw + n + i));
+            if (p.out_fp32) {
+              float* dst = reinterpret_cast<float*>(p.Y) + (size_t)row * p.N + n;
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
+            } else {
+              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.Y) + (size_t)row * p.N + n;
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(y[i], y[i + 1]), h1 = __floats2bfloat162_rn(y[i + 2], y[i + 3]);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(y[i + 4], y[i + 5]), h3 = __floats2bfloat162_rn(y[i + 6], y[i + 7]);
+                *reinterpret_cast<uint4*>(dst + i) =
+                    make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                               *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+              }
+            }
+          }
+        } else if (row < p.M) {
+          float* dst = reinterpret_cast<float*>(p.Y) + (size_t)row * p.N + n;
           if (n + 32 <= p.N) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -243,7 +282,9 @@ typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void
                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+// A K-major operand [outer][inner] of 2-byte (BF16) or 1-byte elements, 128-byte
+// swizzle, boxes of 128 bytes of K by box_outer rows.
+bool map_kmajor(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer, bool s8) {
   static EncodeFn fn = nullptr;
   if (!fn) {
     void* f = nullptr;
@@ -253,28 +294,45 @@ bool map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
       return false;
     fn = reinterpret_cast<EncodeFn>(f);
   }
+  const uint64_t esz = s8 ? 1 : 2;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {PBK, box_outer};
+  cuuint64_t strides[1] = {inner * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(PROW / esz), box_outer};
   cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, s8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool S8>
+cudaError_t launch_dense(const DenseMaps& tm, const DenseParams& p, int num_sms, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(dense_gemm_kernel<S8>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  if (e != cudaSuccess) return e;
+  const int ntiles = ((p.M + PBM - 1) / PBM) * ((p.N + PBN - 1) / PBN);
+  const int sms = num_sms > 0 ? num_sms : 148;
+  dense_gemm_kernel<S8><<<ntiles < sms ? ntiles : sms, P_THREADS, P_SMEM, st>>>(tm, p);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_pca(const PcaLaunch& a, cudaStream_t st) {
-  PcaMaps tm;
+cudaError_t launch_gemm_w8a8(const GemmLaunch& a, cudaStream_t st) {
+  DenseMaps tm;
   memset(&tm, 0, sizeof(tm));
-  if (!map_bf16(&tm.a, a.x, a.K, a.rows, PBM) || !map_bf16(&tm.b, a.vt, a.K, a.K, PBN)) return cudaErrorInvalidValue;
-  PcaParams p{a.rows, a.K, a.K, a.y, a.status, a.wait_ns};
-  cudaError_t e = cudaFuncSetAttribute(pca_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+  if (!map_kmajor(&tm.a, a.a_codes, a.K, a.M, PBM, true) || !map_kmajor(&tm.b, a.w_codes, a.K, a.N, PBN, true))
+    return cudaErrorInvalidValue;
+  DenseParams p{a.M, a.N, a.K, a.Y, a.out_fp32, a.a_scale, a.w_scale, a.status, a.wait_ns};
+  return launch_dense<true>(tm, p, a.num_sms, st);
+}
+
+cudaError_t launch_pca(const PcaLaunch& a, cudaStream_t st) {
+  DenseMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  if (!map_kmajor(&tm.a, a.x, a.K, a.rows, PBM, false) || !map_kmajor(&tm.b, a.vt, a.K, a.K, PBN, false))
+    return cudaErrorInvalidValue;
+  DenseParams p{a.rows, a.K, a.K, a.y, 1, nullptr, nullptr, a.status, a.wait_ns};
+  cudaError_t e = launch_dense<false>(tm, p, a.num_sms, st);
   if (e != cudaSuccess) return e;
-  const int ntiles = ((a.rows + PBM - 1) / PBM) * ((a.K + PBN - 1) / PBN);
-  const int sms = a.num_sms > 0 ? a.num_sms : 148;
-  pca_gemm_kernel<<<ntiles < sms ? ntiles : sms, P_THREADS, P_SMEM, st>>>(tm, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.weight)
     pca_quant_kernel<true><<<a.rows, 128, 0, st>>>(a.y, a.rows, a.K, a.r, a.coef, a.codes, a.scale);
   else

@@ -192,3 +192,37 @@ def test_w4a8_layer(name, M, N):
     o4 = orc.rotate_quantize(inputs.bf16_to_f32(X), orc.INT4, w.block, o_sign, o_perm)
     Y4 = orc.reference_gemm(orc.INT4, orc.INT4, o4["q"], o4["scale"], ow["q"], ow["scale"])
     assert H.rel_fro(Yref, ref) < H.rel_fro(Y4, ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,M,N", [("c1", 256, 1152), ("c2", 300, 640), ("c3", 130, 288)])
+def test_w8a8_layer(name, M, N):
+    # TR-DQ's W8A8 setting (Tables 1-5; section 3.1: per-token activations,
+    # per-channel weights): both operands 8-bit, one dense kind::i8 GEMM
+    w = inputs.WORKLOADS[name]
+    X = inputs.activations(w, M=M)
+    W = inputs.weights(w, N=N)
+    o_sign, o_perm = orc.make_rotation(w.K, w.block, 0)
+    _, _, rot = rq.rq_make_rotation(w.K, w.block, 0)
+    r1 = _dev(rot)
+    ga = _quant2(rq.INT8, X, w.block, r1, None)
+    gw = _quant2(rq.INT8, W, w.block, r1, None, weight=True)
+    oa = orc.rotate_quantize(inputs.bf16_to_f32(X), orc.INT8, w.block, o_sign, o_perm)
+    ow = orc.rotate_quantize(inputs.bf16_to_f32(W), orc.INT8, w.block, o_sign, o_perm, weight_rows=True)
+    H.assert_quant_equal(ga, oa, "activations")
+    H.assert_quant_equal(gw, ow, "weights")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Yf = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    Yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for Y, f in ((Yf, 1), (Yb, 0)):
+        rq.rq_w4a4_linear(rq.INT8, rq.INT8, M, N, w.K, ga["codes_t"], ga["scale_t"], None, gw["codes_t"],
+                          gw["scale_t"], None, None, None, None, None, Y, f, status)
+        assert rq.rq_read_status(status)[0] == 0
+    Yref = orc.reference_gemm(orc.INT8, orc.INT8, oa["q"], oa["scale"], ow["q"], ow["scale"])
+    assert H.rel_fro(Yf.cpu().numpy(), Yref) <= TOL
+    assert torch.equal(Yb, Yf.to(torch.bfloat16))
+    # 8-bit weights track x W^T more closely than 4-bit ones
+    ref = inputs.bf16_to_f32(X).astype(np.float64) @ inputs.bf16_to_f32(W).astype(np.float64).T
+    o4 = orc.rotate_quantize(inputs.bf16_to_f32(W), orc.INT4, w.block, o_sign, o_perm, weight_rows=True)
+    Y4 = orc.reference_gemm(orc.INT8, orc.INT4, oa["q"], oa["scale"], o4["q"], o4["scale"])
+    assert H.rel_fro(Yref, ref) < H.rel_fro(Y4, ref)

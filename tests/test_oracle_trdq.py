@@ -1,12 +1,14 @@
 """Pins for the oracle's TR-DQ pieces (CPU): the zigzag permutation and the
 double block rotation (TR-DQ: Time-Rotation Diffusion Quantization, section
-3.2, Eq. 9) and asymmetric per-token INT4 (section 3.1, Eq. 1-3)."""
+3.2, Eq. 9), asymmetric per-token INT4 (section 3.1, Eq. 1-3) and the 8-bit
+per-token / per-channel settings."""
 import math
 
 import numpy as np
 import pytest
 
 from oracle import rq_oracle as orc
+from rotated_bit_post_b200 import inputs
 
 F32 = np.float32
 
@@ -116,3 +118,23 @@ def test_int8_hand_cases_and_bound():
     Y = orc.reference_gemm(orc.INT8, orc.INT4, q, s, qw, sw)
     B = qw.astype(np.float64) * np.repeat(sw.T.astype(np.float64), 128, axis=1)
     assert np.allclose(Y, (q * s[:, None].astype(np.float64)) @ B.T, rtol=1e-12)
+
+
+def test_w8a8_weight_rows_per_channel():
+    # W8A8 (TR-DQ section 3.1: per-channel weights): one scale per rotated
+    # weight row, amax/127, and the layer tracks x W^T closer than W4A8 does
+    w = inputs.WORKLOADS["c1"]
+    sign, perm = orc.make_rotation(w.K, w.block, 0)
+    X = inputs.bf16_to_f32(inputs.activations(w, M=64))
+    W = inputs.bf16_to_f32(inputs.weights(w, N=96))
+    ow = orc.rotate_quantize(W, orc.INT8, w.block, sign, perm, weight_rows=True)
+    yw = orc.rotate(W, sign, perm, w.block)
+    assert ow["scale"].shape == (96,)
+    assert np.array_equal(ow["scale"], (np.max(np.abs(yw), axis=1) / np.float32(127)).astype(np.float32))
+    assert np.all(np.abs(ow["q"].astype(np.float64) * ow["scale"][:, None] - yw) <= ow["scale"][:, None] * 0.5 * (1 + 1e-6))
+    oa = orc.rotate_quantize(X, orc.INT8, w.block, sign, perm)
+    o4 = orc.rotate_quantize(W, orc.INT4, w.block, sign, perm, weight_rows=True)
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    e8 = np.linalg.norm(orc.reference_gemm(orc.INT8, orc.INT8, oa["q"], oa["scale"], ow["q"], ow["scale"]) - ref)
+    e4 = np.linalg.norm(orc.reference_gemm(orc.INT8, orc.INT4, oa["q"], oa["scale"], o4["q"], o4["scale"]) - ref)
+    assert e8 < 0.5 * e4
