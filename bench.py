@@ -587,7 +587,7 @@ def layer_result(L, args, t_step, t_k1, t_k2, clocks, dist, world, sms):
         # (the split/quantize pass that follows is in the same time)
         pf = pca_flops(w)
         k1_tf = pf / (k1_ms * 1e-3) / 1e12
-        k1_roof = {"kernel": "pca_gemm_kernel + pca_quant_kernel (rq_pca_rotate_quantize_act)", "bound": "tensor",
+        k1_roof = {"kernel": "dense_gemm_kernel<BF16> + pca_quant_kernel (rq_pca_rotate_quantize_act)", "bound": "tensor",
                    "achieved": k1_tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": k1_tf / pk["bf16_tflops"],
                    "peak_source": pk["source"] + " bf16 burst (MEASURED_PEAKS bf16_tflops)",
                    "algorithmic_per_launch": f"{pf:.4g} FLOP (2MK^2); HBM {kb} B at {k1_gbs:.0f} GB/s "

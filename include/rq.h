@@ -193,7 +193,8 @@ rq_status rq_quantize_weights(int32_t fmt, const uint16_t* W, int32_t N, int32_t
  *     the random signs of `rot` (its permutation must be the identity) and an
  *     orthonormal Walsh-Hadamard transform per natural block, P = rot2's
  *     permutation (its sign bits must be clear), R2 a second per-block
- *     transform.  Without rot2 the rotation is the one of `rot`, as in
+ *     transform; K <= 8192 (the kernel keeps the once-rotated row in shared
+ *     memory as FP32).  Without rot2 the rotation is the one of `rot`, as in
  *     rq_rotate_quantize_act.
  *   - fmt RQ_INT8: 8-bit activations for the W4A8 setting (Tables 1-5): inv =
  *     127 / amax, q = clamp(rne(y inv), -127, 127), one byte per code (codes

@@ -8,7 +8,8 @@ the product: the two share only the seeded input generators.
 What it computes, in plain numpy, step by step as the pages state it:
 
 * the randomized permuted block-Hadamard (RPBH) rotation R = BlockDiag(H_b/sqrt b) P D
-  (OrbitQuant abstract: "randomized permuted block-Hadamard (RPBH) rotation";
+  (OrbitQuant abstract: random signs, a permutation and block Hadamard
+  transforms, the RPBH rotation;
   TR-DQ section 3.2, Eq. 8: block-diagonal rotation with K = C_in / 2^n blocks;
   TR-DQ section 3.2: a permutation is itself orthogonal);
 * folding the rotation into the weights, W' = W R^T, so that it cancels inside
@@ -21,6 +22,11 @@ What it computes, in plain numpy, step by step as the pages state it:
     NVFP4 on Blackwell);
 * the DiRotQ low-rank branch: r PCA coefficients kept in BF16 and the residual
   quantized (DiRotQ abstract);
+* DiRotQ's full PCA rotation y = x V, its first r coordinates in BF16 and the
+  rest quantized (DiRotQ abstract);
+* TR-DQ's zigzag permutation and double block rotation (section 3.2, Eq. 9),
+  asymmetric per-token INT4 (section 3.1, Eq. 1-3) and the 8-bit per-token /
+  per-channel quantizer of the W4A8 and W8A8 settings (section 3.1, Tables 1-5);
 * the FP64 reference GEMM over the dequantized values.
 
 Readings taken where the pages are silent:

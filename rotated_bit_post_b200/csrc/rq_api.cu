@@ -71,6 +71,7 @@ rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows,
   if (K % 128) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of 128", K);
   if (fmt == RQ_NVFP4 && U && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 with the low-rank branch needs K %% 256 == 0 (K=%d)", K);
   if (rot2 && U) return fail(RQ_ERR_UNSUPPORTED, "the double rotation runs without the low-rank branch");
+  if (rot2 && K > 8192) return fail(RQ_ERR_UNSUPPORTED, "the double rotation supports K <= 8192 (got %d)", K);
   if (fmt == RQ_INT4A && !zp) return fail(RQ_ERR_INVALID_ARG, "asymmetric INT4 needs a zero-point output");
   if ((fmt == RQ_INT4A || fmt == RQ_INT8) && U) return fail(RQ_ERR_UNSUPPORTED, "format %d runs without the low-rank branch", fmt);
   if ((rot2 && !aligned16(rot2)) || (zp && !aligned16(zp))) return fail(RQ_ERR_ALIGNMENT, "rot2 / zero point not 16-byte aligned");
@@ -128,6 +129,8 @@ rq_status run_k1(int32_t fmt, bool weight, const uint16_t* X, int32_t rows, int3
   a.wait_ns = g_wait_ns.load();
   a.inject_tx = g_inject_tx.load();
   cudaError_t e = rq::launch_k1(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue)   // no kernel configuration fits this format, K and block
+    return fail(RQ_ERR_UNSUPPORTED, "format %d with K=%d, block=%d: no kernel configuration fits", fmt, K, block);
   if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "rotate/quantize launch failed: %s", cudaGetErrorString(e));
   return ok();
 }
