@@ -323,7 +323,10 @@ rq_status rq_pca_rotate_quantize_act_noalloc(const uint16_t* X, int32_t M, int32
  *          symmetric Lloyd-Max codebook is; otherwise RQ_ERR_UNSUPPORTED.
  *   c, L, r  [device] low-rank branch (r == 32) or NULL / 0.
  *   Y      [device, M x N] FP32 (out_fp32 = 1) or BF16 (out_fp32 = 0).
- *   Shapes: M >= 1, N % 32 == 0, K % 128 == 0 (K % 256 == 0 for NVFP4).
+ *   Shapes: M >= 0, N >= 1 (INT4 weights: N % 4 == 0, their group scales are
+ *          copied 16 bytes at a time), K % 128 == 0 (K % 256 == 0 for NVFP4).
+ *          BF16 rows of Y go out through TMA stores when N % 8 == 0 (16-byte
+ *          aligned rows) and through masked element stores otherwise.
  */
 rq_status rq_w4a4_linear(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N, int32_t K, const uint8_t* a_codes,
                          const float* a_scale, const uint8_t* a_bscale, const uint8_t* w_codes,

@@ -325,7 +325,8 @@ static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N,
                        (a_fmt == RQ_LM16 && w_fmt == RQ_LM4) || (a_fmt == RQ_NVFP4 && w_fmt == RQ_NVFP4);
   if (!pair_ok) return fail(RQ_ERR_UNSUPPORTED, "format pair (%d, %d) not supported", a_fmt, w_fmt);
   if (M < 0 || N <= 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape M=%d N=%d K=%d", M, N, K);
-  if (N % 32) return fail(RQ_ERR_INVALID_ARG, "N=%d must be a multiple of 32", N);
+  if (w_fmt == RQ_INT4 && N % 4)   // the group scales of a tile are copied 16 bytes at a time
+    return fail(RQ_ERR_INVALID_ARG, "INT4 weights need N %% 4 == 0 (N=%d)", N);
   if (K % 128) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of 128", K);
   if (a_fmt == RQ_NVFP4 && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs K %% 256 == 0 (K=%d)", K);
   if (!a_codes || !a_scale || !w_codes || !w_scale || !Y) return fail(RQ_ERR_INVALID_ARG, "null pointer");

@@ -253,8 +253,9 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       break;
     }
     // ------------------------------------------------------------ restage
-    for (int u = threadIdx.x; u < nr * (K / 8); u += blockDim.x) {
-      const int r = u / (K / 8), j = u - r * (K / 8);
+    // (row, 16-byte unit) advanced by the block's stride without a division per step
+    const int K8 = K / 8, dr = (int)blockDim.x / K8, dj = (int)blockDim.x - dr * K8;
+    for (int r = (int)threadIdx.x / K8, j = (int)threadIdx.x - r * K8; r < nr;) {
       const uint4 d = *reinterpret_cast<const uint4*>(land + (size_t)r * K * 2 + (size_t)j * 16);
       const uint32_t sw = sgnw[j];
       uint32_t* dst = reinterpret_cast<uint32_t*>(stg + (size_t)r * P + (size_t)j * 16);
@@ -262,6 +263,12 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       dst[1] = d.y ^ ((sw << 1) & 0x80008000u);
       dst[2] = d.z ^ ((sw << 2) & 0x80008000u);
       dst[3] = d.w ^ ((sw << 3) & 0x80008000u);
+      j += dj;
+      r += dr;
+      if (j >= K8) {
+        j -= K8;
+        ++r;
+      }
     }
     __syncthreads();
     if (*abort_flag) break;

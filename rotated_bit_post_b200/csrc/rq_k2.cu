@@ -148,11 +148,13 @@ __device__ __forceinline__ void fma_s32x2(float& r0, float& r1, float w0, float 
       : "r"(x0 + 0x4B400000u), "r"(x1 + 0x4B400000u), "f"(w0), "f"(w1), "f"(12582912.0f));
 }
 
-// Store 32 consecutive outputs of one row (FP32 or BF16), masked to n < N.
+// Store 32 consecutive outputs of one row (FP32 or BF16), masked to n < N;
+// 16-byte stores where the row and the chunk are whole and aligned (N a
+// multiple of 4 FP32 or 8 BF16 values), element stores otherwise.
 __device__ __forceinline__ void store_row32(void* Y, int out_fp32, int N, int m, int n0, const float (&v)[32]) {
   if (out_fp32) {
     float* dst = reinterpret_cast<float*>(Y) + (size_t)m * N + n0;
-    if (n0 + 32 <= N) {
+    if (n0 + 32 <= N && (N & 3) == 0) {
 #pragma unroll
       for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
     } else {
@@ -168,7 +170,7 @@ __device__ __forceinline__ void store_row32(void* Y, int out_fp32, int N, int m,
       __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
       w[i] = *reinterpret_cast<uint32_t*>(&h);
     }
-    if (n0 + 32 <= N) {
+    if (n0 + 32 <= N && (N & 7) == 0) {
 #pragma unroll
       for (int i = 0; i < 16; i += 4)
         *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
@@ -1412,7 +1414,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
     return launch(gemm_nvf4_kernel<128>, Nvf4Plan<128>::BYTES, grid, NVF4_THREADS, tm, gp, st);
   }
   const bool w2 = a.w_fmt == RQ_FMT_LM4;
-  if (!a.out_fp32) {
+  if (!a.out_fp32 && a.N % 8 == 0) {   // (the map's row pitch must be a multiple of 16 bytes)
     // BF16 output through 32 x 32 boxes (the epilogue's TMA stores)
     ok &= make_map_2d(&tm.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, a.N, a.M, (uint64_t)a.N * 2, 32, 32,
                       CU_TENSOR_MAP_SWIZZLE_64B);

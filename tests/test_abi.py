@@ -83,8 +83,8 @@ def test_argument_errors_are_host_side(L):
     assert code == 1  # 2-bit codes are for weights only
     code = L.rq_w4a4_linear(rq.INT4, rq.LM16, 4, 32, 128, *([None] * 10), 0, None, 1, None, None)
     assert code == 2
-    code = L.rq_w4a4_linear(rq.INT4, rq.INT4, 4, 40, 128, *([None] * 10), 0, None, 1, None, None)
-    assert code == 1 and "N=40" in rq.rq_last_error()
+    code = L.rq_w4a4_linear(rq.INT4, rq.INT4, 4, 42, 128, *([None] * 10), 0, None, 1, None, None)
+    assert code == 1 and "N=42" in rq.rq_last_error()   # INT4 weights: N % 4 == 0
     # misaligned device pointer
     p = ctypes.c_void_p(0x1008)
     code = L.rq_rotate_quantize_act(rq.INT4, p, 4, 1152, 128, p, None, None, 0, None, p, p, None, None, None)

@@ -104,3 +104,28 @@ def test_other_block_sizes(name, block):
     # K / 2^n blocks); blocks above 128 span several threads of the kernel
     w = dataclasses.replace(inputs.WORKLOADS[name], block=block)
     run_layer(w, 97, 256)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,N", [("c3", 77), ("c5", 300), ("c5", 1), ("c4", 99), ("c1", 100), ("c2", 200),
+                                    ("c3", 455)])
+def test_any_n(name, N):
+    # output widths that are not multiples of the tile's 32-column chunks:
+    # masked element stores (N % 8 != 0: BF16 rows are not 16-byte aligned,
+    # so no TMA stores), the last weight rows zero-filled by the loads; INT4
+    # weights (group scales copied 16 bytes at a time) take N % 4 == 0
+    run_layer(inputs.WORKLOADS[name], 130, N)
+
+
+@pytest.mark.gpu
+def test_int4_weights_reject_n_not_multiple_of_4():
+    w = inputs.WORKLOADS["c1"]
+    Y = torch.empty((8, 6), dtype=torch.float32, device="cuda")
+    codes_a = torch.zeros((8, w.K // 2), dtype=torch.uint8, device="cuda")
+    codes_w = torch.zeros((6, w.K // 2), dtype=torch.uint8, device="cuda")
+    sa = torch.zeros(8, dtype=torch.float32, device="cuda")
+    sw = torch.zeros((w.K // 128, 6), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(rq.RQError, match="N % 4"):
+        rq.rq_w4a4_linear(rq.INT4, rq.INT4, 8, 6, w.K, codes_a, sa, None, codes_w, sw, None, None, None, None, None,
+                          Y, 1, status)

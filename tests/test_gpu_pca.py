@@ -74,11 +74,13 @@ def _check_split(g, y, r, weight):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name,M,N,K", [("c2", 300, 320, 1152), ("c1", 129, 256, 1152), ("c2", 64, 160, 512)])
+@pytest.mark.parametrize("name,M,N,K", [("c2", 300, 320, 1152), ("c1", 129, 256, 1152), ("c2", 64, 160, 512),
+                                        ("c2", 4096, 256, 1152)])
 def test_pca_layer(name, M, N, K):
     """Activations and weights through the full rotation, then the 4-bit GEMM
-    with the rank-32 BF16 term; ragged M (a partial 128-row tile) and K not a
-    multiple of the 256-wide output tile."""
+    with the rank-32 BF16 term; ragged M (a partial 128-row tile), K not a
+    multiple of the 256-wide output tile, and the PixArt fc1 token count,
+    whose product runs on 128-wide tiles (two even rounds on 148 SMs)."""
     import dataclasses
     w = dataclasses.replace(inputs.WORKLOADS[name], K=K)
     r = 32
