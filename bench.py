@@ -52,12 +52,14 @@ MMA_FLOP_PER_CLK_SM = {"fp8": 2 * 128 * 256 * 32 / 128, "s8": 2 * 128 * 256 * 32
 NOMINAL_RATIO_TO_BF16 = {"fp8": 2, "s8": 2, "fp4": 4}
 
 # DRAM bytes (read + write) per launch of each kernel from a 1-pass ncu capture
-# of the current kernels at the full sizes; None where the kernel changed after
-# the last capture.  The capture command and per-kernel figures are kept with
-# the other ncu summaries under profiles/.
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the current kernels at the
+# full sizes, L2 flushed before each step as in the timed run; None where the
+# kernel changed after the last capture.  Outputs still dirty in L2 when a
+# kernel ends are written back later and not counted here.  The capture command
+# and per-kernel figures are kept with the other ncu summaries under profiles/.
 TRAFFIC = {
-    "k2": {"c1": None, "c2": None, "c3": None, "c4": None, "c5": None},
-    "k1": {"c1": None, "c2": None, "c3": None, "c4": None, "c5": None},
+    "k2": {"c1": 0.9e6, "c2": 5.8e6, "c3": 52.2e6, "c4": 53.6e6, "c5": 1170.8e6, "c2p": 5.8e6},
+    "k1": {"c1": 0.6e6, "c2": 9.6e6, "c3": 28.4e6, "c4": 122.9e6, "c5": 232.5e6, "c2p": 31.0e6},
 }
 
 
@@ -592,7 +594,7 @@ def layer_result(L, args, t_step, t_k1, t_k2, clocks, dist, world, sms):
                    "peak_source": pk["source"] + " bf16 burst (MEASURED_PEAKS bf16_tflops)",
                    "algorithmic_per_launch": f"{pf:.4g} FLOP (2MK^2); HBM {kb} B at {k1_gbs:.0f} GB/s "
                                              f"(2K + 8K + K/2 + 4 + 2r per token, + 2K^2 for V)",
-                   "traffic": None}
+                   "traffic": None if args.tokens else TRAFFIC["k1"].get(w.name)}
     k2_roof = {"kernel": "gemm kernel of rq_w4a4_linear", "bound": "tensor", "achieved": k2_tflops,
                "peak": tp["peak"], "unit": "TFLOP/s", "frac": k2_tflops / tp["peak"],
                "peak_source": tp["peak_source"], "alt_peaks": tp["alt_peaks"],
