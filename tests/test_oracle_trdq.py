@@ -15,8 +15,8 @@ F32 = np.float32
 
 def test_zigzag_hand_dealt():
     # K = 8 channels, blocks of 2 -> 4 blocks; ranked: 4 (9), 6 (7), 1 (5),
-    # 2 (3), 5 (1), 7 (0.3), 3 (0.2), 0 (0.1).  Round 0 deals blocks 0..3 their
-    # first slot, round 1 deals blocks 3..0 their second slot.
+    # 2 (3), 5 (1), 7 (0.3), 3 (0.2), 0 (0.1).  The first pass deals blocks
+    # 0..3 their first slot, the second pass blocks 3..0 their second slot.
     mag = [0.1, 5, 3, 0.2, 9, 1, 7, 0.3]
     assert list(orc.zigzag_permutation(mag, 2)) == [4, 0, 6, 3, 1, 7, 2, 5]
     # equal magnitudes rank by channel index
