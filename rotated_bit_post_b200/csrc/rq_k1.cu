@@ -764,6 +764,8 @@ cudaError_t launch_k1_t(const K1Launch& a, cudaStream_t st) {
   if (R > 24 && !PROJ) R = 24;
   // (the coefficient and residual mappings cover at most 32 rows)
   if (PROJ) R = min(min(R, 32), max(1, (a.rows + sms - 1) / sms));
+  // few rows: smaller groups, so that every resident CTA gets some
+  else R = min(R, max(1, (a.rows + (IPW == 1 ? 2 : 1) * sms - 1) / ((IPW == 1 ? 2 : 1) * sms)));
   size_t smem = k1_smem_bytes(R, a.K, nblk, PROJ, ngrp, p.lut_n);
   // two CTAs per SM for the single-pass variant
   const size_t cap = PROJ ? 232448 : IPW == 1 ? 110 * 1024 : 200 * 1024;
