@@ -145,9 +145,10 @@ rq_status rq_pca_basis(const uint16_t* calib, int32_t n, int32_t K, int32_t r, u
  *          K % 128 == 0; with U: block 128, 256 or 512 and, for NVFP4, K % 256 == 0.
  *   rot    [device, K] signed permutation from rq_make_rotation.
  *   boundaries [host, levels-1] FP32 codebook boundaries (RQ_LM16), else NULL.
- *   U, r   [device, K x r] BF16 PCA basis and its rank (r == 32, K <= 3072:
+ *   U, r   [device, K x r] BF16 PCA basis and its rank (r in {8, 16, 24, 32}, K <= 3072:
  *          U^T is staged whole in shared memory), or NULL / 0.
- *          With U: c = bf16(x U) (FP32, sequential over k) is written to c_out
+ *          With U: c = bf16(x U) (FP32: a sequential chain over each 128-channel
+ *          chunk in k order, the chunk sums added in order) is written to c_out
  *          and the residual x - c U^T is what gets rotated and quantized.
  *   c_out  [device, M x r] BF16 or NULL.
  *   codes  [device, M x K/2] packed nibbles.
@@ -172,8 +173,8 @@ rq_status rq_rotate_quantize_act(int32_t fmt, const uint16_t* X, int32_t M, int3
  *   fmt    RQ_INT4 (one scale per 128 rotated coordinates) | RQ_LM16 | RQ_LM4 |
  *          RQ_NVFP4.
  *   W      [device, N x K] BF16.
- *   U, r, L_out  optional (r == 32, K <= 3072): L = bf16(W U) [device, N x r]
- *          (FP32, sequential over k) for the low-rank branch
+ *   U, r, L_out  optional (r in {8, 16, 24, 32}, K <= 3072): L = bf16(W U) [device, N x r]
+ *          (FP32, the same chunked order) for the low-rank branch
  *          (the full row is still what gets quantized).
  *   codes  [device, N x K/2] (RQ_LM4: N x K/4).
  *   scale  [device] RQ_INT4: [K/128][N] group-major; otherwise [N].
@@ -242,7 +243,7 @@ rq_status rq_quantize_weights2(int32_t fmt, const uint16_t* W, int32_t N, int32_
  *   Vt     [device, K x K] BF16, row n = column n of V (V orthogonal: the
  *          PCA basis of the calibration tokens, all K eigenvectors, dominant
  *          first).
- *   r      0 <= r <= K (the GEMM's low-rank term takes r == 32).
+ *   r      0 <= r <= K (the GEMM's low-rank term takes r in {8, 16, 24, 32}).
  *   workspace [device, M x K] FP32, caller-allocated scratch: y is written
  *          there (and may be read back; it is the rotated activation).
  *   c_out  [device, M x r] BF16 (may be NULL when r == 0).
@@ -321,7 +322,7 @@ rq_status rq_pca_rotate_quantize_act_noalloc(const uint16_t* X, int32_t M, int32
  *          Read during the argument checks.  A 16-entry table must be
  *          symmetric (entry 7-m = entry 8+m with the sign bit set), which the
  *          symmetric Lloyd-Max codebook is; otherwise RQ_ERR_UNSUPPORTED.
- *   c, L, r  [device] low-rank branch (r == 32) or NULL / 0.
+ *   c, L, r  [device] low-rank branch (r in {8, 16, 24, 32}; M x r and N x r BF16) or NULL / 0.
  *   Y      [device, M x N] FP32 (out_fp32 = 1) or BF16 (out_fp32 = 0).
  *   Shapes: M >= 0, N >= 1 (INT4 weights: N % 4 == 0, their group scales are
  *          copied 16 bytes at a time), K % 128 == 0 (K % 256 == 0 for NVFP4).

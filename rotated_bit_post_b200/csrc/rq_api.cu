@@ -80,7 +80,8 @@ rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows,
     return fail(RQ_ERR_INVALID_ARG, "codebook format needs boundaries");
   if (fmt == RQ_NVFP4 && !bscale) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs block_scale");
   if (U) {
-    if (r != 32) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r == 32 (got %d)", r);
+    if (r < 8 || r > 32 || r % 8)
+      return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r in {8, 16, 24, 32} (got %d)", r);
     if (K > 3072) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports K <= 3072 (got %d)", K);
     if (!coef) return fail(RQ_ERR_INVALID_ARG, "U given without a coefficient output");
     if (!aligned16(U) || !aligned16(coef)) return fail(RQ_ERR_ALIGNMENT, "U / coefficient output not 16-byte aligned");
@@ -344,7 +345,8 @@ static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N,
     return fail(RQ_ERR_UNSUPPORTED, "16-level activation table is not symmetric (entry 7-m must be -(entry 8+m))");
   if (w_fmt == RQ_LM16 && !symmetric16(w_lut))
     return fail(RQ_ERR_UNSUPPORTED, "16-level weight table is not symmetric (entry 7-m must be -(entry 8+m))");
-  if (c && r != 32) return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r == 32 (got %d)", r);
+  if (c && (r < 8 || r > 32 || r % 8))
+    return fail(RQ_ERR_UNSUPPORTED, "low-rank branch supports r in {8, 16, 24, 32} (got %d)", r);
   if (c && (a_fmt == RQ_INT8 || a_fmt == RQ_INT4A))
     return fail(RQ_ERR_UNSUPPORTED, "the low-rank branch runs with 4-bit activations");
   const void* ptrs[] = {a_codes, a_scale, w_codes, w_scale, Y, a_bscale, w_bscale, c, L};

@@ -235,11 +235,14 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
 
   if constexpr (PROJ) {
     // stage U^T (row j holds U[0..K-1][j]) and the signed permutation once per
-    // CTA, while the first rows stream in
+    // CTA, while the first rows stream in.  A rank below 32 is padded with zero
+    // columns: their coefficients are 0 and their products in the residual are
+    // zeros, so every chain's result is that of the first r terms.
     const int KP = ut_pitch(K);
+    const int rq8 = p.r / 8;   // 16-byte words per row of U
     for (int t = threadIdx.x; t < K * 4; t += K1_THREADS) {
       const int k = t >> 2, q = t & 3;
-      const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)k * 32) + q);
+      const uint4 w4 = q < rq8 ? __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)k * p.r) + q) : make_uint4(0, 0, 0, 0);
       const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(K1_THREADS, IPW == 1 ? 2 : 1) k1_rotate_quanti
           float s = cp[0];
           for (int t = 1; t < nch; ++t) s = __fadd_rn(s, cp[t * 32]);
           const uint16_t h = __bfloat16_as_ushort(__float2bfloat16_rn(s));
-          p.coef[(size_t)(r0 + row) * 32 + j] = h;
+          if (j < p.r) p.coef[(size_t)(r0 + row) * p.r + j] = h;
           negc[row * 32 + j] = -bf16_bits_to_f32(h);
         }
       }

@@ -129,3 +129,15 @@ def test_int4_weights_reject_n_not_multiple_of_4():
     with pytest.raises(rq.RQError, match="N % 4"):
         rq.rq_w4a4_linear(rq.INT4, rq.INT4, 8, 6, w.K, codes_a, sa, None, codes_w, sw, None, None, None, None, None,
                           Y, 1, status)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,r,K", [("c2", 8, None), ("c2", 16, None), ("c2", 24, None), ("c3", 16, None),
+                                      ("c4", 16, 3072)])
+def test_other_ranks(name, r, K):
+    # ranks below 32 (multiples of 8): the projection pads U with zero columns
+    # and the GEMM's low-rank tiles are zero-filled past r by the loads
+    w = dataclasses.replace(inputs.WORKLOADS[name], rank=r)
+    if K:
+        w = dataclasses.replace(w, K=K)
+    run_layer(w, 130, 256)

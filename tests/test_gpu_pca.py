@@ -110,7 +110,7 @@ def test_pca_layer(name, M, N, K):
 @pytest.mark.gpu
 @pytest.mark.parametrize("r", [0, 8, 200])
 def test_pca_split_widths(r):
-    """Other widths of the BF16 part (no GEMM: its low-rank term takes r = 32)."""
+    """Other widths of the BF16 part (no GEMM: its low-rank term takes r <= 32)."""
     w = inputs.WORKLOADS["c1"]
     X = inputs.activations(w, M=70)
     V = _basis_bits(w, w.K)
