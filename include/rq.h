@@ -141,8 +141,11 @@ rq_status rq_pca_basis(const uint16_t* calib, int32_t n, int32_t K, int32_t r, u
  * (OrbitQuant abstract: only a forward rotation on the activations remains at
  * run time; TR-DQ section 3.2: dynamic per-token ranges computed online.)
  *   fmt    RQ_INT4 | RQ_LM16 | RQ_NVFP4.
- *   X      [device, M x K] BF16.     M >= 1.  K % block == 0, K <= 16384,
- *          K % 128 == 0; with U: block 128, 256 or 512 and, for NVFP4, K % 256 == 0.
+ *   X      [device, M x K] BF16.     M >= 1.  K % block == 0, K <= 16384;
+ *          K % 64 == 0 for RQ_LM16 and RQ_NVFP4 (their packed rows stay whole
+ *          16-byte units for the GEMM's tensor maps), K % 128 == 0 for RQ_INT4
+ *          (weight groups of 128) and with U; with U: block 128, 256 or 512
+ *          and, for NVFP4, K % 256 == 0.
  *   rot    [device, K] signed permutation from rq_make_rotation.
  *   boundaries [host, levels-1] FP32 codebook boundaries (RQ_LM16), else NULL.
  *   U, r   [device, K x r] BF16 PCA basis and its rank (r in {8, 16, 24, 32}, K <= 3072:
@@ -172,7 +175,8 @@ rq_status rq_rotate_quantize_act(int32_t fmt, const uint16_t* X, int32_t M, int3
  * the rotation absorbed into the weights).
  *   fmt    RQ_INT4 (one scale per 128 rotated coordinates) | RQ_LM16 | RQ_LM4 |
  *          RQ_NVFP4.
- *   W      [device, N x K] BF16.
+ *   W      [device, N x K] BF16.  K as for rq_rotate_quantize_act (RQ_LM4:
+ *          K % 64 == 0).
  *   U, r, L_out  optional (r in {8, 16, 24, 32}, K <= 3072): L = bf16(W U) [device, N x r]
  *          (FP32, the same chunked order) for the low-rank branch
  *          (the full row is still what gets quantized).
@@ -325,7 +329,10 @@ rq_status rq_pca_rotate_quantize_act_noalloc(const uint16_t* X, int32_t M, int32
  *   c, L, r  [device] low-rank branch (r in {8, 16, 24, 32}; M x r and N x r BF16) or NULL / 0.
  *   Y      [device, M x N] FP32 (out_fp32 = 1) or BF16 (out_fp32 = 0).
  *   Shapes: M >= 0, N >= 1 (INT4 weights: N % 4 == 0, their group scales are
- *          copied 16 bytes at a time), K % 128 == 0 (K % 256 == 0 for NVFP4).
+ *          copied 16 bytes at a time).  K % 64 == 0 for the codebook and NVFP4
+ *          pairs (a last K step that is only partly inside K is zero-filled by
+ *          the loads and only its MMAs inside K are issued); K % 128 == 0 when
+ *          the weights are INT4 or INT8 (whole 128-wide groups).
  *          BF16 rows of Y go out through TMA stores when N % 8 == 0 (16-byte
  *          aligned rows) and through masked element stores otherwise.
  */

@@ -68,7 +68,11 @@ rq_status check_rows_call(int32_t fmt, bool weight, const void* X, int32_t rows,
     return fail(RQ_ERR_UNSUPPORTED, "block %d with the low-rank branch: 128, 256 or 512", block);
   if (K % block) return fail(RQ_ERR_INVALID_ARG, "K=%d is not a multiple of block=%d", K, block);
   if (K > 16384) return fail(RQ_ERR_UNSUPPORTED, "K=%d exceeds 16384", K);
-  if (K % 128) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of 128", K);
+  // codebook and NVFP4 rows need K % 64 (their packed rows stay whole 16-byte
+  // units for the GEMM's tensor maps); INT4 groups, 8-bit codes, the low-rank
+  // branch and the double rotation need K % 128
+  const bool k64 = (fmt == RQ_LM16 || fmt == RQ_LM4 || fmt == RQ_NVFP4) && !U && !rot2;
+  if (K % (k64 ? 64 : 128)) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of %d", K, k64 ? 64 : 128);
   if (fmt == RQ_NVFP4 && U && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 with the low-rank branch needs K %% 256 == 0 (K=%d)", K);
   if (rot2 && U) return fail(RQ_ERR_UNSUPPORTED, "the double rotation runs without the low-rank branch");
   if (rot2 && K > 8192) return fail(RQ_ERR_UNSUPPORTED, "the double rotation supports K <= 8192 (got %d)", K);
@@ -328,8 +332,10 @@ static rq_status linear_impl(int32_t a_fmt, int32_t w_fmt, int32_t M, int32_t N,
   if (M < 0 || N <= 0 || K <= 0) return fail(RQ_ERR_INVALID_ARG, "bad shape M=%d N=%d K=%d", M, N, K);
   if (w_fmt == RQ_INT4 && N % 4)   // the group scales of a tile are copied 16 bytes at a time
     return fail(RQ_ERR_INVALID_ARG, "INT4 weights need N %% 4 == 0 (N=%d)", N);
-  if (K % 128) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of 128", K);
-  if (a_fmt == RQ_NVFP4 && K % 256) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs K %% 256 == 0 (K=%d)", K);
+  // codebook and NVFP4 codes: K % 64 (a ragged last K step issues only its
+  // MMAs inside K); INT4 and 8-bit weights: whole 128-wide groups
+  const bool k64 = a_fmt == RQ_LM16 || a_fmt == RQ_NVFP4;
+  if (K % (k64 ? 64 : 128)) return fail(RQ_ERR_INVALID_ARG, "K=%d must be a multiple of %d", K, k64 ? 64 : 128);
   if (!a_codes || !a_scale || !w_codes || !w_scale || !Y) return fail(RQ_ERR_INVALID_ARG, "null pointer");
   if (a_fmt == RQ_NVFP4 && (!a_bscale || !w_bscale)) return fail(RQ_ERR_INVALID_ARG, "NVFP4 needs block scales");
   if (a_fmt == RQ_LM16 && (!a_lut || !w_lut)) return fail(RQ_ERR_INVALID_ARG, "codebook formats need LUTs");

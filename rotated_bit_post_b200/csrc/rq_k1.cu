@@ -832,11 +832,12 @@ cudaError_t launch_k1_fmt(const K1Launch& a, cudaStream_t st) {
 
 cudaError_t launch_k1(const K1Launch& a, cudaStream_t st) {
   // the rows-as-lanes kernel: for what only it does (double rotation, INT4A,
-  // INT8, the weight code sums, blocks outside 128-512) and where its layout pays: whole rows of 32
+  // INT8, the weight code sums, blocks outside 128-512, K an odd multiple of
+  // 64) and where its layout pays: whole rows of 32
   // tokens per warp (K <= 1536) and enough row groups to fill the GPU twice;
   // measured on B200: Wan-like K = 1536 169 us against 186 us, while the
   // PixArt-width, FLUX QKV and FLUX down-projection layers ran faster here
-  const bool only_r = a.rot2 || a.fmt == RQ_FMT_INT4A || a.fmt == RQ_FMT_INT8 || a.wz ||
+  const bool only_r = a.rot2 || a.fmt == RQ_FMT_INT4A || a.fmt == RQ_FMT_INT8 || a.wz || a.K % 128 ||
                       (a.block != 128 && a.block != 256 && a.block != 512);
   const int sms = a.num_sms > 0 ? a.num_sms : 148;
   const bool r_pays = a.K <= 1536 && a.block <= 128 && a.rows >= 32 * 2 * sms;

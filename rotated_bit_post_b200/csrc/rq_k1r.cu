@@ -21,14 +21,14 @@
 //    its FP32 output stored at an odd-word row pitch, gathered again through
 //    the zigzag permutation]
 //   phase A: a warp's lanes are R rows x F segments; a thread owns one segment
-//     of 128 consecutive rotated coordinates of one row, gathered through the
+//     of 128 consecutive rotated coordinates of one row (64 when K is an odd
+//     multiple of 64), gathered through the
 //     permutation table (byte offsets) into registers; butterflies of blocks up
 //     to 128 run in registers (blocks of 256-1024: T = b/128 threads, the last
 //     log2 T stages through __shfl_xor_sync); y = v * fp32(1/sqrt b); per-block
 //     pairwise sums of squares or per-segment maxima go to shared memory
 //   phase B: every thread derives its row's scale from the partials in the
-//     same order, quantizes its 128 values, packs them and stores 64 (or 32)
-//     bytes of codes.
+//     same order, quantizes its segment, packs it and stores its codes.
 //
 // FP32 contract (bit-exact against the CPU oracle): explicit round-to-nearest-
 // even operations, no contraction; packed f32x2 operations round each lane
@@ -49,8 +49,9 @@ namespace {
 
 constexpr int R_THREADS = 384;     // 12 warps
 constexpr int R_LUT_MAX = 1536;    // codebook cells
-constexpr int SEG = 128;           // rotated coordinates per thread
-constexpr int TS = SEG + 4;        // table stride per segment (entries), breaks bank aliasing
+// rotated coordinates per thread (SEG): 128, or 64 for rows with K % 128 != 0
+// (blocks up to 64; codebook and NVFP4 codes); the gather table's stride per
+// segment is SEG + 4 entries, which breaks bank aliasing
 
 struct __align__(16) K1RParams {
   const uint16_t* x;       // rows x K, BF16 bits
@@ -104,13 +105,13 @@ __device__ __forceinline__ void mul2s(float& v0, float& v1, float s) {
       : "+f"(v0), "+f"(v1)
       : "f"(s));
 }
-// Butterflies of the thread's 128 registers: blocks of min(b, 128), stages in
+// Butterflies of the thread's SEG registers: blocks of min(b, SEG), stages in
 // ascending stride; stride 1 pairs share a register pair (scalar), strides 2+
-// run as packed pairs; then the cross-thread strides 128 .. b/2 with the lanes
+// run as packed pairs; then the cross-thread strides SEG .. b/2 with the lanes
 // l ^ m of the same block (lower lane v + o, upper lane o - v, both exact
 // single roundings).
-template <int B>
-__device__ __forceinline__ void fwht128(float (&v)[SEG], int part) {
+template <int B, int SEG>
+__device__ __forceinline__ void fwht_seg(float (&v)[SEG], int part) {
   constexpr int IN = B < SEG ? B : SEG;
   constexpr int T = B > SEG ? B / SEG : 1;
 #pragma unroll
@@ -142,14 +143,14 @@ __device__ __forceinline__ void fwht128(float (&v)[SEG], int part) {
 // tree), evaluated depth first so that only the partial sums of the open
 // subtrees are live; every subtree of size `in` (the block, at most 128) is
 // written to out[its first index / in].
-template <int I, int N>
+template <int SEG, int I, int N>
 struct SqTree {
   static __device__ __forceinline__ float run(const float (&v)[SEG], int in, float* out) {
     float r;
     if constexpr (N == 1) {
       r = __fmul_rn(v[I], v[I]);
     } else {
-      r = __fadd_rn(SqTree<I, N / 2>::run(v, in, out), SqTree<I + N / 2, N / 2>::run(v, in, out));
+      r = __fadd_rn(SqTree<SEG, I, N / 2>::run(v, in, out), SqTree<SEG, I + N / 2, N / 2>::run(v, in, out));
     }
     if constexpr (N >= 16) {   // blocks are at least 16 wide
       if (N == in) out[I / N] = r;
@@ -158,8 +159,11 @@ struct SqTree {
   }
 };
 
-template <int FMT, bool WEIGHT, int B>
+template <int FMT, bool WEIGHT, int B, int SEG>
 __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant__ K1RParams p) {
+  static_assert(SEG == 128 || (B <= 64 && (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4 || FMT == RQ_FMT_NVFP4)),
+                "64-wide segments carry codebook and NVFP4 rows with blocks up to 64");
+  constexpr int TS = SEG + 4;
   constexpr int T = B > SEG ? B / SEG : 1;        // threads per Hadamard block (<= F)
   const int F = p.F;
   const bool DBL = p.dbl != 0;
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
 #pragma unroll
         for (int e = 0; e < SEG; ++e) v[e] = bf16_bits_to_f32(src[e]);
       }
-      fwht128<B>(v, part);
+      fwht_seg<B, SEG>(v, part);
 #pragma unroll
       for (int e = 0; e < SEG; e += 2) mul2s(v[e], v[e + 1], p.inv_sqrt_b);
       if (live) {
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
         }
       }
     }
-    fwht128<B>(v, part);
+    fwht_seg<B, SEG>(v, part);
 #pragma unroll
     for (int e = 0; e < SEG; e += 2) mul2s(v[e], v[e + 1], p.inv_sqrt_b);
 
@@ -334,7 +338,7 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       // blocks up to 128: their trees straight to the partials; larger blocks:
       // the 128-wide subtrees added across the block's threads (xor 1, 2, 4)
       // (a thread that is not live passes block width 0: nothing is written)
-      float ss = SqTree<0, SEG>::run(v, (live && B <= SEG) ? B : 0, pt + rl * pstride + seg * NBT);
+      float ss = SqTree<SEG, 0, SEG>::run(v, (live && B <= SEG) ? B : 0, pt + rl * pstride + seg * NBT);
 #pragma unroll
       for (int m = 1; m < T; m <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, m));
       if (B > SEG && live && part == 0) pt[rl * pstride + seg / T] = ss;
@@ -441,7 +445,7 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       // one byte per code (two's complement), 32 codes per pair of 16-byte stores
       uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * K + (size_t)seg * SEG);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < SEG / 32; ++c) {
         uint32_t w[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) w[j] = 0u;
@@ -455,9 +459,9 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
         dst[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
     } else if constexpr (FMT == RQ_FMT_INT4 || FMT == RQ_FMT_INT4A) {
-      uint32_t pk[16];
+      uint32_t pk[SEG / 8];
 #pragma unroll
-      for (int w = 0; w < 16; ++w) pk[w] = 0u;
+      for (int w = 0; w < SEG / 8; ++w) pk[w] = 0u;
       if constexpr (FMT == RQ_FMT_INT4) {
 #pragma unroll
         for (int e = 0; e < SEG; ++e) {
@@ -476,14 +480,14 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       }
       uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 2) + (size_t)seg * (SEG / 2));
 #pragma unroll
-      for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      for (int c = 0; c < SEG / 32; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
     } else if constexpr (FMT == RQ_FMT_LM16 || FMT == RQ_FMT_LM4) {
       // t = u * 2^s, exactly 2^s * fp32(v * inv) (the scaling is exact): the
       // cell of t and one compare against the cell's scaled boundary
       const float mlt_s = __fmul_rn(mlt, __int_as_float((127 + p.lut_shift) << 23));
       const uint32_t gbias = 0x4B400000u + (uint32_t)p.lut_gmin;
       const uint32_t nmax = (uint32_t)p.lut_n - 1u;
-      constexpr int NW32 = FMT == RQ_FMT_LM16 ? 16 : 8;
+      constexpr int NW32 = FMT == RQ_FMT_LM16 ? SEG / 8 : SEG / 16;
       uint32_t pk[NW32];
 #pragma unroll
       for (int w = 0; w < NW32; ++w) pk[w] = 0u;
@@ -502,17 +506,17 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       if constexpr (FMT == RQ_FMT_LM16) {
         uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 2) + (size_t)seg * (SEG / 2));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        for (int c = 0; c < SEG / 32; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       } else {
         uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 4) + (size_t)seg * (SEG / 4));
 #pragma unroll
-        for (int c = 0; c < 2; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        for (int c = 0; c < SEG / 64; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
-    } else {   // NVFP4: eight 16-element groups
-      uint32_t pk[16];
+    } else {   // NVFP4: SEG / 16 groups of 16 elements
+      uint32_t pk[SEG / 8];
       uint32_t sbw[2] = {0u, 0u};
 #pragma unroll
-      for (int gq = 0; gq < 8; ++gq) {
+      for (int gq = 0; gq < SEG / 16; ++gq) {
         float* u = v + 16 * gq;
         float m16 = 0.f;
 #pragma unroll
@@ -539,20 +543,20 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       }
       uint4* dst = reinterpret_cast<uint4*>(p.codes + (size_t)row * (K / 2) + (size_t)seg * (SEG / 2));
 #pragma unroll
-      for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      for (int c = 0; c < SEG / 32; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       // block scales kb .. kb+3 (kb % 4 == 0) are four adjacent bytes of the tile layout
       const int kb = seg * (SEG / 16);
       *reinterpret_cast<uint32_t*>(p.bscale + sf_off(row, kb, K)) = sbw[0];
-      *reinterpret_cast<uint32_t*>(p.bscale + sf_off(row, kb + 4, K)) = sbw[1];
+      if constexpr (SEG == 128) *reinterpret_cast<uint32_t*>(p.bscale + sf_off(row, kb + 4, K)) = sbw[1];
     }
   }
 }
 
 // ------------------------------------------------------------------ host side
-size_t k1r_smem(int RW, int K, int S, bool dbl, int nblk, int nwarps, int npart, int lut_n) {
+size_t k1r_smem(int RW, int K, int S, int ts, bool dbl, int nblk, int nwarps, int npart, int lut_n) {
   size_t off = (size_t)RW * K * 2 + (size_t)RW * (2 * K + 4) + (dbl ? (size_t)RW * (4 * K + 4) : 0);
   off = (off + 15) & ~(size_t)15;
-  off += (size_t)S * TS * 4;
+  off += (size_t)S * ts * 4;
   off += (size_t)(K / 8) * 4;
   off += (size_t)2 * RW * (nblk > S ? nblk : S) * npart * 4;
   off = (off + 15) & ~(size_t)15;
@@ -605,7 +609,7 @@ bool build_cells(K1RParams& p, const float* bnd, int nbnd, int K, bool sign_magn
   return false;
 }
 
-template <int FMT, bool WEIGHT, int B>
+template <int FMT, bool WEIGHT, int B, int SEG>
 cudaError_t launch_r(const K1Launch& a, cudaStream_t st) {
   constexpr int T = B > SEG ? B / SEG : 1;
   K1RParams p{};
@@ -640,7 +644,7 @@ cudaError_t launch_r(const K1Launch& a, cudaStream_t st) {
   size_t smem = 0;
   for (int f = 1; f <= 16; f *= 2) {
     const int nw = (S + f - 1) / f;
-    const size_t sm = k1r_smem(32 / f, a.K, S, p.dbl != 0, a.K / a.block, nw, npart, p.lut_n);
+    const size_t sm = k1r_smem(32 / f, a.K, S, SEG + 4, p.dbl != 0, a.K / a.block, nw, npart, p.lut_n);
     if (f >= T && nw <= R_THREADS / 32 && sm <= 232448) {
       F = f;
       smem = sm;
@@ -652,7 +656,7 @@ cudaError_t launch_r(const K1Launch& a, cudaStream_t st) {
   p.R = 32 / F;
   p.ngroups = (a.rows + p.R - 1) / p.R;
   const int nwarps = (S + F - 1) / F;
-  auto kern = k1r_kernel<FMT, WEIGHT, B>;
+  auto kern = k1r_kernel<FMT, WEIGHT, B, SEG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int sms = a.num_sms > 0 ? a.num_sms : 148;
@@ -665,7 +669,11 @@ cudaError_t launch_r(const K1Launch& a, cudaStream_t st) {
 
 bool k1r_supports(const K1Launch& a) {
   if (a.U) return false;
-  if (a.K % SEG) return false;
+  if (a.K % 64) return false;
+  // 64-wide segments: codebook and NVFP4 codes with blocks up to 64, one rotation
+  if (a.K % 128 && (a.block > 64 || a.rot2 || a.wz ||
+                    (a.fmt != RQ_FMT_LM16 && a.fmt != RQ_FMT_LM4 && a.fmt != RQ_FMT_NVFP4)))
+    return false;
   if (a.rot2 && a.K > 8192) return false;   // the FP32 row copy of the double rotation
   switch (a.block) {
     case 16: case 32: case 64: case 128: case 256: case 512: case 1024: return true;
@@ -674,23 +682,37 @@ bool k1r_supports(const K1Launch& a) {
 }
 
 namespace {
+// rows whose K is an odd multiple of 64 (blocks up to 64): 64-wide segments
+template <int BS>
+cudaError_t launch_r_t64(const K1Launch& a, cudaStream_t st) {
+  if constexpr (BS <= 64) {
+    switch (a.fmt) {
+      case RQ_FMT_LM16: return a.weight ? launch_r<RQ_FMT_LM16, true, BS, 64>(a, st) : launch_r<RQ_FMT_LM16, false, BS, 64>(a, st);
+      case RQ_FMT_LM4: return a.weight ? launch_r<RQ_FMT_LM4, true, BS, 64>(a, st) : cudaErrorInvalidValue;
+      case RQ_FMT_NVFP4: return a.weight ? launch_r<RQ_FMT_NVFP4, true, BS, 64>(a, st) : launch_r<RQ_FMT_NVFP4, false, BS, 64>(a, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int BS>
 cudaError_t launch_r_t(const K1Launch& a, cudaStream_t st) {
+  if (a.K % 128) return launch_r_t64<BS>(a, st);
   if (a.weight) {
     switch (a.fmt) {
-      case RQ_FMT_INT4: return launch_r<RQ_FMT_INT4, true, BS>(a, st);
-      case RQ_FMT_LM16: return launch_r<RQ_FMT_LM16, true, BS>(a, st);
-      case RQ_FMT_LM4: return launch_r<RQ_FMT_LM4, true, BS>(a, st);
-      case RQ_FMT_NVFP4: return launch_r<RQ_FMT_NVFP4, true, BS>(a, st);
+      case RQ_FMT_INT4: return launch_r<RQ_FMT_INT4, true, BS, 128>(a, st);
+      case RQ_FMT_LM16: return launch_r<RQ_FMT_LM16, true, BS, 128>(a, st);
+      case RQ_FMT_LM4: return launch_r<RQ_FMT_LM4, true, BS, 128>(a, st);
+      case RQ_FMT_NVFP4: return launch_r<RQ_FMT_NVFP4, true, BS, 128>(a, st);
     }
     return cudaErrorInvalidValue;
   }
   switch (a.fmt) {
-    case RQ_FMT_INT4: return launch_r<RQ_FMT_INT4, false, BS>(a, st);
-    case RQ_FMT_INT4A: return launch_r<RQ_FMT_INT4A, false, BS>(a, st);
-    case RQ_FMT_INT8: return launch_r<RQ_FMT_INT8, false, BS>(a, st);
-    case RQ_FMT_LM16: return launch_r<RQ_FMT_LM16, false, BS>(a, st);
-    case RQ_FMT_NVFP4: return launch_r<RQ_FMT_NVFP4, false, BS>(a, st);
+    case RQ_FMT_INT4: return launch_r<RQ_FMT_INT4, false, BS, 128>(a, st);
+    case RQ_FMT_INT4A: return launch_r<RQ_FMT_INT4A, false, BS, 128>(a, st);
+    case RQ_FMT_INT8: return launch_r<RQ_FMT_INT8, false, BS, 128>(a, st);
+    case RQ_FMT_LM16: return launch_r<RQ_FMT_LM16, false, BS, 128>(a, st);
+    case RQ_FMT_NVFP4: return launch_r<RQ_FMT_NVFP4, false, BS, 128>(a, st);
   }
   return cudaErrorInvalidValue;
 }

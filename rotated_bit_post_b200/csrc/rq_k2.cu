@@ -41,6 +41,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 
 #include "rq_internal.h"
 #include "rq_ptx.cuh"
@@ -61,6 +62,7 @@ struct __align__(64) TMaps {
 
 struct __align__(16) GemmParams {
   int M, N, K;
+  int nk128;                // 128-wide K tiles, ceil(K / 128)
   int a_fmt, w_fmt;
   const float* a_scale;
   const float* w_scale;     // INT4: [K/128][N]; else [N]
@@ -461,7 +463,12 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
   float* sc_slots = reinterpret_cast<float*>(smem + P::OFF_SC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = p.K / 128;                // 128-wide K tiles == INT4 groups
+  // 128-wide K tiles (== INT4 groups); codebook codes may end in a half tile
+  // (K % 128 == 64): its zero-filled upper half is expanded but never multiplied.
+  // (The count comes from the host: derived from K in the kernel, the codebook
+  // loop measured ~0.8% slower.)
+  const int nk = p.nk128;
+  const int kk_last = (p.K - (nk - 1) * 128) / 32;   // 32-code MMAs in the last K tile (2 or 4)
   constexpr bool grouped = GROUPED;
   const bool lr = P::LR && p.has_lr;
   // PAIR: the two CTAs of a cluster share 256 x BN tiles; CTA `crank` takes
@@ -596,7 +603,10 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
       if constexpr (WIDE) {
         // single accumulators (all 512 columns): the first MMA of a tile into
         // either half waits until the epilogue has drained that half of the
-        // previous tile
+        // previous tile.  Two copies of the loop: whole last K tiles (the
+        // common case, no per-step test) or half ones (K % 128 == 64)
+        auto wide_loop = [&](auto half_tail) {
+        constexpr bool HALF = decltype(half_tail)::value;
         for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
           for (int kt = 0; kt < nk; ++kt, ++kc) {
             const int s = kc % P::SE;
@@ -611,10 +621,12 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
                 if (!ok) break;
                 tc_fence_after();
               }
+              const int kkn = (HALF && kt == nk - 1) ? 2 : 4;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                umma_f8_2(tmem + h * 256, smem_desc(a + kk * 32, 16, 1024, 2),
-                          smem_desc(b + h * 128 * 128 + kk * 32, 16, 1024, 2), idesc, (kt == 0 && kk == 0) ? 0u : 1u);
+                if (!HALF || kk < kkn)
+                  umma_f8_2(tmem + h * 256, smem_desc(a + kk * 32, 16, 1024, 2),
+                            smem_desc(b + h * 128 * 128 + kk * 32, 16, 1024, 2), idesc, (kt == 0 && kk == 0) ? 0u : 1u);
             }
             if (!ok) break;
             tc_commit2_mc(&eempty[s], 0x3);   // the stage is free in both CTAs
@@ -622,6 +634,11 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           if (!ok) break;
           tc_commit2_mc(&accfull[0], 0x3);
         }
+        };
+        if (kk_last == 4)
+          wide_loop(std::false_type{});
+        else
+          wide_loop(std::true_type{});
       }
       for (int tile = tile0; tile < ntiles && ok && !WIDE; tile += tstep, ++tc) {
         const uint32_t ab = tc & 1;
@@ -649,8 +666,10 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           const uint32_t a = A8 ? sbase + P::OFF_PA + (kc % P::SP) * P::PA : sbase + P::OFF_EA + s * P::EA;
           const uint32_t b = sbase + P::OFF_EB + s * P::EB;
           const bool fresh = grouped || kt == 0;
+          const int kkn = kt == nk - 1 ? kk_last : 4;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
+            if (kk >= kkn) break;
             if constexpr (GROUPED)
               umma_i8(tmem + buf * 128, smem_desc(a + kk * 32, 16, 1024, 2), smem_desc(b + kk * 32, 16, 1024, 2),
                       idesc, (fresh && kk == 0) ? 0u : 1u);
@@ -1079,7 +1098,9 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
   float* sc_slots = reinterpret_cast<float*>(smem + P::OFF_SC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = p.K / 256;
+  // 256-wide K steps; the last may hold 1-3 of its four 64-wide scale tiles
+  // (K % 64 == 0): only those are copied and multiplied
+  const int nk = (p.K + 255) / 256;
   const int ktiles64 = p.K / 64;          // scale tiles per 128 rows
   const bool lr = P::LR && p.has_lr;
   const int nN = (p.N + BN - 1) / BN, nM = (p.M + BM - 1) / BM;
@@ -1128,14 +1149,15 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
           const int s = kc % P::S;
           if (kc >= P::S && !mbar_wait(&empty[s], ((kc / P::S) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
           uint8_t* st = smem + s * P::STAGE;
-          mbar_expect_tx(&full[s], P::PA + P::PB + P::SA + nb_valid * 2048 + (kc == 0 ? p.inject_tx : 0u));
+          const uint32_t sfb = (uint32_t)min(4, ktiles64 - kt * 4) * 512;   // scale bytes per 128 rows
+          mbar_expect_tx(&full[s], P::PA + P::PB + sfb + nb_valid * sfb + (kc == 0 ? p.inject_tx : 0u));
           tma_load_2d(st, &tm.a, kt * 128, m0, &full[s]);
           tma_load_2d(st + P::PA, &tm.b, kt * 128, n0, &full[s]);
-          // 4 scale chunks (k tiles of 64) x 512 B, contiguous in the K1 layout
-          bulk_g2s(st + P::PA + P::PB, sfa_src + (size_t)kt * 4 * 512, 2048, &full[s]);
+          // up to 4 scale chunks (k tiles of 64) x 512 B, contiguous in the K1 layout
+          bulk_g2s(st + P::PA + P::PB, sfa_src + (size_t)kt * 4 * 512, sfb, &full[s]);
           for (int nb = 0; nb < nb_valid; ++nb)
             bulk_g2s(st + P::PA + P::PB + P::SA + nb * 2048,
-                     p.w_bscale + ((size_t)(n0 / 128 + nb) * ktiles64 + (size_t)kt * 4) * 512, 2048, &full[s]);
+                     p.w_bscale + ((size_t)(n0 / 128 + nb) * ktiles64 + (size_t)kt * 4) * 512, sfb, &full[s]);
         }
         if (lr) {   // after the K tiles (see the codebook kernel)
           if (tc > 0 && !mbar_wait(lrsmem_empty, (tc - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
@@ -1173,9 +1195,11 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
           tc_fence_after();
           const uint32_t st = sbase + s * P::STAGE;
           const uint32_t t_sfa = tmem + 256 + sl * SF_COLS, t_sfb = t_sfa + 16;
+          const int kkn = min(4, ktiles64 - kt * 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_nvf4(tmem + ab * BN, smem_desc(st + kk * 32, 16, 1024, 2), smem_desc(st + P::PA + kk * 32, 16, 1024, 2),
+            if (kk < kkn)
+              umma_nvf4(tmem + ab * BN, smem_desc(st + kk * 32, 16, 1024, 2), smem_desc(st + P::PA + kk * 32, 16, 1024, 2),
                       idesc, t_sfa + kk * 4, t_sfb + kk * (BN / 32), (kt > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
           tc_commit(&sfempty[sl]);
@@ -1379,6 +1403,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t st, const char** why) 
   memset(&tm, 0, sizeof(tm));
   GemmParams gp{};
   gp.M = a.M; gp.N = a.N; gp.K = a.K;
+  gp.nk128 = (a.K + 127) / 128;
   gp.a_fmt = a.a_fmt; gp.w_fmt = a.w_fmt;
   gp.a_scale = a.a_scale; gp.w_scale = a.w_scale;
   gp.a_bscale = a.a_bscale; gp.w_bscale = a.w_bscale;

@@ -107,6 +107,39 @@ def test_other_block_sizes(name, block):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("name,K,block,N", [("c3", 192, 64, 256), ("c3", 64, 64, 300), ("c5", 320, 32, 640),
+                                            ("c5", 64, 16, 256), ("c4", 192, 64, 256), ("c4", 320, 16, 384),
+                                            ("c4", 64, 64, 128)])
+def test_k_odd_multiple_of_64(name, K, block, N):
+    # codebook and NVFP4 rows whose K is an odd multiple of 64: 64-wide
+    # segments in the activation kernel; in the GEMM the last K step is partly
+    # zero-filled by the loads and only its MMAs (and, for NVFP4, its scale
+    # tiles) inside K are issued
+    w = dataclasses.replace(inputs.WORKLOADS[name], K=K, block=block)
+    run_layer(w, 130, N)
+
+
+@pytest.mark.gpu
+def test_k_multiple_of_128_where_required():
+    # INT4 groups and the low-rank branch keep K % 128 == 0
+    K = 192
+    X = torch.zeros((4, K), dtype=torch.int16, device="cuda")
+    _, _, rot = rq.rq_make_rotation(K, 64, 0)
+    rot_t = torch.from_numpy(rot).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b = rq.act_buffers(rq.INT4, 4, K)
+    with pytest.raises(rq.RQError, match="multiple of 128"):
+        rq.rq_rotate_quantize_act(rq.INT4, X, 64, rot_t, None, None, None, b["codes"], b["scale"], None, status)
+    U = torch.zeros((K, 32), dtype=torch.int16, device="cuda")
+    c = torch.empty((4, 32), dtype=torch.int16, device="cuda")
+    cb = rq.rq_make_codebook(K, 16)
+    b = rq.act_buffers(rq.LM16, 4, K)
+    with pytest.raises(rq.RQError):
+        rq.rq_rotate_quantize_act(rq.LM16, X, 64, rot_t, cb["boundaries_f32"], U, c, b["codes"], b["scale"], None,
+                                  status)
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("name,N", [("c3", 77), ("c5", 300), ("c5", 1), ("c4", 99), ("c1", 100), ("c2", 200),
                                     ("c3", 455)])
 def test_any_n(name, N):
