@@ -288,8 +288,7 @@ __device__ __forceinline__ void tmem_ld_wait_regs16(uint32_t (&r)[16]) {
 }
 
 // y for four consecutive columns: acc * (s_a * s_w), on packed FP32 pairs
-__device__ __forceinline__ void scale4(const uint32_t* a, const float* sw, float sa, float (&y)[4]) {
-  const float4 w4 = *reinterpret_cast<const float4*>(sw);
+__device__ __forceinline__ void scale4w(const uint32_t* a, float4 w4, float sa, float (&y)[4]) {
   float s0 = sa, s1 = sa, s2 = sa, s3 = sa;
   mul2_f32(s0, s1, w4.x, w4.y);
   mul2_f32(s2, s3, w4.z, w4.w);
@@ -300,20 +299,24 @@ __device__ __forceinline__ void scale4(const uint32_t* a, const float* sw, float
   mul2_f32(y[0], y[1], s0, s1);
   mul2_f32(y[2], y[3], s2, s3);
 }
+__device__ __forceinline__ void scale4(const uint32_t* a, const float* sw, float sa, float (&y)[4]) {
+  scale4w(a, *reinterpret_cast<const float4*>(sw), sa, y);
+}
 
-// Epilogue of the 256 x 512 pair tiles: this warp drains 256 accumulator
+// Epilogue of the 256 x 512 pair tiles: this warp drains 16 * NCH accumulator
 // columns of its 32 token rows.  BF16 output: 16 columns at a time, the TMEM
 // load of the next 16 in flight while these are scaled and written to one of
 // this warp's two 2 KB staging buffers; every 32 columns go out as one TMA
 // store.  FP32 output (used for verification): 32 columns at a time, stored
 // straight to global memory, the same FP32 values.
-__device__ __forceinline__ void epi_half_wide(const GemmParams& p, const CUtensorMap* ymap, uint32_t tacc,
+template <int NCH>
+__device__ __forceinline__ void epi_cols_wide(const GemmParams& p, const CUtensorMap* ymap, uint32_t tacc,
                                               const float* sw, float sa, int row, int n0, int row0, uint32_t stg,
                                               uint32_t& stc) {
   const int lane = threadIdx.x & 31;
   if (!p.tma_store) {
 #pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
+    for (int ch = 0; ch < NCH / 2; ++ch) {
       uint32_t a[32];
       tmem_ld32(tacc + ch * 32, a);
       tmem_ld_wait();
@@ -331,9 +334,14 @@ __device__ __forceinline__ void epi_half_wide(const GemmParams& p, const CUtenso
   uint32_t acc[2][16];
   tmem_ld16(tacc, acc[0]);
 #pragma unroll
-  for (int hc = 0; hc < 16; ++hc) {
+  for (int hc = 0; hc < NCH; ++hc) {
+    // this chunk's weight scales, read before the wait so that their latency
+    // overlaps it (the wait orders every memory access around it)
+    float4 w4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w4[i] = *reinterpret_cast<const float4*>(sw + hc * 16 + 4 * i);
     tmem_ld_wait_regs16(acc[hc & 1]);
-    if (hc + 1 < 16) tmem_ld16(tacc + (hc + 1) * 16, acc[(hc + 1) & 1]);
+    if (hc + 1 < NCH) tmem_ld16(tacc + (hc + 1) * 16, acc[(hc + 1) & 1]);
     const uint32_t buf = stg + (stc & 1u) * 2048u;
     if ((hc & 1) == 0 && stc >= 2) {   // the store two boxes back must have read this buffer
       if (lane == 0) bulk_wait_group_read<1>();
@@ -342,8 +350,8 @@ __device__ __forceinline__ void epi_half_wide(const GemmParams& p, const CUtenso
 #pragma unroll
     for (int c = 0; c < 2; ++c) {   // 8 columns -> one 16-byte shared store of BF16
       float y0[4], y1[4];
-      scale4(acc[hc & 1] + 8 * c, sw + hc * 16 + 8 * c, sa, y0);
-      scale4(acc[hc & 1] + 8 * c + 4, sw + hc * 16 + 8 * c + 4, sa, y1);
+      scale4w(acc[hc & 1] + 8 * c, w4[2 * c], sa, y0);
+      scale4w(acc[hc & 1] + 8 * c + 4, w4[2 * c + 1], sa, y1);
       __nv_bfloat162 h0 = __floats2bfloat162_rn(y0[0], y0[1]), h1 = __floats2bfloat162_rn(y0[2], y0[3]);
       __nv_bfloat162 h2 = __floats2bfloat162_rn(y1[0], y1[1]), h3 = __floats2bfloat162_rn(y1[2], y1[3]);
       const int cc = 2 * (hc & 1) + c;   // 16-byte column of the 32 x 32 box
@@ -487,8 +495,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     // PAIR: efull / accempty of the even CTA count both CTAs' warps; eempty and
     // accfull take one multicast commit arrival in each CTA
     for (int i = 0; i < P::SE; ++i) { mbar_init(&efull[i], PAIR ? 2 * NXW : NXW); mbar_init(&eempty[i], 1); }
-    // WIDE: accempty[h] counts the warps draining half h (four per CTA)
-    constexpr int ACC_ARRIVALS = WIDE ? 2 * (NEPI / 2) : PAIR ? 2 * NEPI : NEPI;
+    // PAIR: every epilogue warp of both CTAs (WIDE: per 256-column half)
+    constexpr int ACC_ARRIVALS = PAIR ? 2 * NEPI : NEPI;
     for (int i = 0; i < 3; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], ACC_ARRIVALS); }
     mbar_init(lrfull, 1);
     mbar_init(lrsmem_empty, 1);
@@ -605,28 +613,57 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         // either half waits until the epilogue has drained that half of the
         // previous tile.  Two copies of the loop: whole last K tiles (the
         // common case, no per-step test) or half ones (K % 128 == 64)
+        static_assert(P::SE >= 2, "the first two K tiles of a tile are held at once");
         auto wide_loop = [&](auto half_tail) {
         constexpr bool HALF = decltype(half_tail)::value;
+        // one K tile's MMAs into half h (TMEM columns h*256 ..) from stage s
+        auto issue = [&](int h, int s, int kt) {
+          const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
+          const int kkn = (HALF && kt == nk - 1) ? 2 : 4;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            if (!HALF || kk < kkn)
+              umma_f8_2(tmem + h * 256, smem_desc(a + kk * 32, 16, 1024, 2),
+                        smem_desc(b + h * 128 * 128 + kk * 32, 16, 1024, 2), idesc, (kt == 0 && kk == 0) ? 0u : 1u);
+        };
         for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
-          for (int kt = 0; kt < nk; ++kt, ++kc) {
+          int kt = 0;
+          if (tc > 0 && nk >= 2) {
+            // the epilogue frees the first half first: its MMAs of the first
+            // two K tiles run while the second half is still being drained
+            const int s0 = kc % P::SE, s1 = (kc + 1) % P::SE;
+            ok = mbar_wait(&efull[s0], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
+                 mbar_wait(&accempty[0], (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            issue(0, s0, 0);
+            ok = mbar_wait(&efull[s1], ((kc + 1) / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            issue(0, s1, 1);
+            ok = mbar_wait(&accempty[1], (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            issue(1, s0, 0);
+            tc_commit2_mc(&eempty[s0], 0x3);   // the stage is free in both CTAs
+            issue(1, s1, 1);
+            tc_commit2_mc(&eempty[s1], 0x3);
+            kt = 2;
+            kc += 2;
+          }
+          for (; kt < nk; ++kt, ++kc) {
             const int s = kc % P::SE;
             ok = mbar_wait(&efull[s], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              if (kt == 0 && tc > 0) {
+              if (kt == 0 && tc > 0) {   // (a single K tile per output tile)
                 ok = mbar_wait(&accempty[h], (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
                 if (!ok) break;
                 tc_fence_after();
               }
-              const int kkn = (HALF && kt == nk - 1) ? 2 : 4;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                if (!HALF || kk < kkn)
-                  umma_f8_2(tmem + h * 256, smem_desc(a + kk * 32, 16, 1024, 2),
-                            smem_desc(b + h * 128 * 128 + kk * 32, 16, 1024, 2), idesc, (kt == 0 && kk == 0) ? 0u : 1u);
+              issue(h, s, kt);
             }
             if (!ok) break;
             tc_commit2_mc(&eempty[s], 0x3);   // the stage is free in both CTAs
@@ -817,19 +854,25 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           ++stc;
         }
       } else if constexpr (WIDE) {
-        const int h = e >> 2;                  // this warp's 256-column half
+        // all eight warps drain the first 256-column half, then the second:
+        // the next tile's MMAs into the first half start while the second
+        // drains.  This warp takes 128 columns of each half.
+        const int part = e >> 2;
         float* sw = sc_slots + (tc & 1) * BN;
         load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid, 32 * NEPI);
         epi_bar_n<32 * NEPI>();
         ok = mbar_wait(&accfull[0], tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
-        epi_half_wide(p, &tm.y, tmem + lane_off + h * 256, sw + h * 256, sa, row, n0 + h * 256, m0 + q * 32, stg,
-                      stc);
-        // this half may take the next tile's first MMA
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(&accempty[h], 0);
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const int c0 = hh * 256 + part * 128;
+          epi_cols_wide<8>(p, &tm.y, tmem + lane_off + c0, sw + c0, sa, row, n0 + c0, m0 + q * 32, stg, stc);
+          // this half may take the next tile's first MMAs
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(&accempty[hh], 0);
+        }
       } else {
         const uint32_t ab = tc & 1;
         float* sw = sc_slots + ab * BN;
