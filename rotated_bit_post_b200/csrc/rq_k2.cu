@@ -226,16 +226,21 @@ __device__ __forceinline__ void epi_chunk_final(const GemmParams& p, uint32_t ta
   tmem_ld32(tacc, acc);
   uint32_t l[32];
   if (lr) tmem_ld32(tlr, l);
-  tmem_ld_wait();
-  float v[32];
+  // s_a * s_w for the 32 columns, formed before the wait (which orders every
+  // memory access around it) so that the scale reads overlap it
+  float s[32];
 #pragma unroll
   for (int i = 0; i < 32; i += 4) {
     const float4 w4 = *reinterpret_cast<const float4*>(sw + i);
-    v[i] = __uint_as_float(acc[i]) * (sa * w4.x);
-    v[i + 1] = __uint_as_float(acc[i + 1]) * (sa * w4.y);
-    v[i + 2] = __uint_as_float(acc[i + 2]) * (sa * w4.z);
-    v[i + 3] = __uint_as_float(acc[i + 3]) * (sa * w4.w);
+    s[i] = sa * w4.x;
+    s[i + 1] = sa * w4.y;
+    s[i + 2] = sa * w4.z;
+    s[i + 3] = sa * w4.w;
   }
+  tmem_ld_wait();
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(acc[i]) * s[i];
   if (lr) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += __uint_as_float(l[i]);
@@ -779,13 +784,18 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           for (int c = 0; c < 2; ++c) {
             uint32_t acc[16];
             tmem_ld16(tmem + lane_off + buf * 128 + h * 32 + c * 16, acc);
-            tmem_ld_wait();
+            // the group scales, read before the wait (which orders every
+            // memory access around it) so that their latency overlaps it
+            float4 w4[4];
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
+            for (int i = 0; i < 4; ++i) w4[i] = *reinterpret_cast<const float4*>(sw + c * 16 + 4 * i);
+            tmem_ld_wait_regs16(acc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
               // S32 partials (|x| <= 256 * 49 * 128 < 2^21) convert to FP32 exactly
-              const float4 w4 = *reinterpret_cast<const float4*>(sw + c * 16 + i);
-              fma_s32x2(run[c * 16 + i], run[c * 16 + i + 1], w4.x, w4.y, acc[i], acc[i + 1]);
-              fma_s32x2(run[c * 16 + i + 2], run[c * 16 + i + 3], w4.z, w4.w, acc[i + 2], acc[i + 3]);
+              fma_s32x2(run[c * 16 + 4 * i], run[c * 16 + 4 * i + 1], w4[i].x, w4[i].y, acc[4 * i], acc[4 * i + 1]);
+              fma_s32x2(run[c * 16 + 4 * i + 2], run[c * 16 + 4 * i + 3], w4[i].z, w4[i].w, acc[4 * i + 2],
+                        acc[4 * i + 3]);
             }
           }
           tc_fence_before();
