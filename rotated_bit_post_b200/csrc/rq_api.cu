@@ -422,6 +422,7 @@ rq_status rq_read_status(const int32_t* status, void* stream, int32_t* code_out)
   e = cudaMemcpy(&v, status, 4, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return fail(RQ_ERR_CUDA, "status read failed: %s", cudaGetErrorString(e));
   if (code_out) *code_out = v;
+  if (v == 0x201) return fail(RQ_ERR_CUDA, "a kernel found its shared memory misaligned (code 0x%x)", v);
   if (v != 0) return fail(RQ_ERR_TIMEOUT, "a kernel gave up a bounded wait (code 0x%x)", v);
   return ok();
 }

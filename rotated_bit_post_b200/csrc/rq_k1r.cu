@@ -252,7 +252,9 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
     const int nr = min(RW, p.rows - r0);
     float* pt = partials + (size_t)(it & 1) * RW * pstride;
     const bool ok = mbar_wait(full, it & 1, p.status, ST_TIMEOUT_LOAD, abort_flag, p.wait_ns);
-    if (!ok) {
+    // one decision for the whole CTA (a thread whose wait ran out must not
+    // leave while another, whose wait just succeeded, heads for a barrier)
+    if (__syncthreads_or(!ok)) {
       if (threadIdx.x == 0) mbar_drain(full, it & 1, p.wait_ns);
       break;
     }

@@ -393,12 +393,16 @@ struct Fp8Plan {
   // PAIR (a CTA pair sharing 256 x 256 tiles): each CTA holds half of the
   // tile's weight rows, so four expanded stages fit.  BN = 512 (CTA pairs
   // only, 256 x 512 tiles): each CTA holds 256 weight rows per stage, two
-  // 128-row halves of the two 256-wide output halves; two or three expanded
-  // stages.
+  // 128-row halves of the two 256-wide output halves; three expanded stages
+  // with two packed ones, which lets the expansion run a stage further ahead
+  // of the MMAs (W2A4 GEMM 769 -> 722 us).  To fit them with 4-bit weights the
+  // tile's weight scales take one slot (refilled after the drain) and the plan
+  // carries no alignment slack: the kernel checks that its dynamic shared
+  // memory starts 1024-byte aligned.
   static constexpr bool WIDE = BN == 512;
   static constexpr int BR = PAIR ? BN / 2 : BN;       // weight rows held by this CTA
-  static constexpr int SP = WIDE ? 3 : PAIR ? 4 : BN == 256 ? (WBITS == 4 ? 4 : 5) : 4;
-  static constexpr int SE = WIDE ? 2 : PAIR ? 4 : BN == 256 ? 2 : 3;
+  static constexpr int SP = WIDE ? 2 : PAIR ? 4 : BN == 256 ? (WBITS == 4 ? 4 : 5) : 4;
+  static constexpr int SE = WIDE ? 3 : PAIR ? 4 : BN == 256 ? 2 : 3;
   static constexpr int STG = WIDE ? 32768 : BN >= 256 ? 16384 : 32768;
   static constexpr int WROW = WBITS == 4 ? 64 : 32;  // packed weight bytes per row per 128-wide K tile
   // A8 (8-bit activations, W4A8): the activation tile arrives as int8 in the
@@ -412,11 +416,13 @@ struct Fp8Plan {
   static constexpr int OFF_C = OFF_EB + SE * EB;
   static constexpr int OFF_L = OFF_C + (LR ? BM * 64 : 0);
   static constexpr int OFF_SC = OFF_L + (LR ? BN * 64 : 0);
-  static constexpr int SCS = BN == 128 ? 12 : 4;               // grouped scale ring depth (BN 128 only)
-  static constexpr int OFF_STG = (OFF_SC + (SCS * BN * 4 > 2 * BN * 4 ? SCS * BN * 4 : 2 * BN * 4) + 1023) & ~1023;
+  static constexpr int SCS = BN == 128 ? 12 : 2;               // grouped scale ring depth (BN 128 only)
+  static constexpr int SC_BYTES = WIDE ? BN * 4 : (SCS * BN * 4 > 2 * BN * 4 ? SCS * BN * 4 : 2 * BN * 4);
+  static constexpr int OFF_STG = (OFF_SC + SC_BYTES + 1023) & ~1023;
   static constexpr int OFF_BAR = OFF_STG + STG;
   static constexpr int NBAR = 2 * SP + 2 * SE + 6 + 4 + 2 * SCS + 1;   // + MMA drain after an abort
-  static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int SLACK = WIDE ? 0 : 1024;                 // alignment slack
+  static constexpr int BYTES = OFF_BAR + NBAR * 8 + 16 + SLACK;
   static_assert(BYTES <= 232448, "shared memory plan exceeds 227 KB");
 };
 
@@ -455,6 +461,14 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
   constexpr int NXT = NXW * 32;                  // expansion threads
   constexpr int NPART = 3;                       // GROUPED partial buffers
   extern __shared__ uint8_t smem_raw[];
+  if constexpr (P::SLACK == 0) {
+    // a plan without slack needs the dynamic shared memory 1024-byte aligned
+    // (every CTA sees the same base, so all leave here together)
+    if (smem_u32(smem_raw) & 1023u) {
+      if (threadIdx.x == 0) atomicCAS(p.status, 0, ST_SMEM_ALIGN);
+      return;
+    }
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
@@ -635,26 +649,27 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           int kt = 0;
           if (tc > 0 && nk >= 2) {
             // the epilogue frees the first half first: its MMAs of the first
-            // two K tiles run while the second half is still being drained
-            const int s0 = kc % P::SE, s1 = (kc + 1) % P::SE;
-            ok = mbar_wait(&efull[s0], (kc / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
-                 mbar_wait(&accempty[0], (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
+            // K tiles (as many as there are expanded stages) run while the
+            // second half is still being drained
+            const int npre = nk < P::SE ? nk : P::SE;
+            ok = mbar_wait(&accempty[0], (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
+            for (int j = 0; j < npre && ok; ++j) {
+              ok = mbar_wait(&efull[(kc + j) % P::SE], ((kc + j) / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag,
+                             p.wait_ns);
+              if (!ok) break;
+              tc_fence_after();
+              issue(0, (kc + j) % P::SE, j);
+            }
             if (!ok) break;
-            tc_fence_after();
-            issue(0, s0, 0);
-            ok = mbar_wait(&efull[s1], ((kc + 1) / P::SE) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns);
-            if (!ok) break;
-            tc_fence_after();
-            issue(0, s1, 1);
             ok = mbar_wait(&accempty[1], (tc - 1) & 1, p.status, ST_TIMEOUT_EPI, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
-            issue(1, s0, 0);
-            tc_commit2_mc(&eempty[s0], 0x3);   // the stage is free in both CTAs
-            issue(1, s1, 1);
-            tc_commit2_mc(&eempty[s1], 0x3);
-            kt = 2;
-            kc += 2;
+            for (int j = 0; j < npre; ++j) {
+              issue(1, (kc + j) % P::SE, j);
+              tc_commit2_mc(&eempty[(kc + j) % P::SE], 0x3);   // the stage is free in both CTAs
+            }
+            kt = npre;
+            kc += npre;
           }
           for (; kt < nk; ++kt, ++kc) {
             const int s = kc % P::SE;
@@ -760,7 +775,10 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     const uint32_t stg = sbase + P::OFF_STG + (uint32_t)e * (GROUPED ? 2048u : 4096u);
     int tc = 0;
     bool ok = true;
-    for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
+    // Without GROUPED the epilogue warps meet at named barriers every tile, so
+    // after an abort they keep walking the tile loop (skipping the work) rather
+    // than leaving it one by one: every warp reaches every barrier.
+    for (int tile = tile0; tile < ntiles && (ok || !GROUPED); tile += tstep, ++tc) {
       const int m0 = (tile / nN) * TM + (int)crank * BM, n0 = (tile % nN) * BN;
       const int row = m0 + q * 32 + lane;
       const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
@@ -868,42 +886,47 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         // the next tile's MMAs into the first half start while the second
         // drains.  This warp takes 128 columns of each half.
         const int part = e >> 2;
-        float* sw = sc_slots + (tc & 1) * BN;
+        // one scale slot: filled once every epilogue warp has finished the
+        // previous tile (the barrier after the drain below)
+        float* sw = sc_slots;
         load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid, 32 * NEPI);
         epi_bar_n<32 * NEPI>();
-        ok = mbar_wait(&accfull[0], tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
-        if (!ok) break;
-        tc_fence_after();
+        ok = ok && mbar_wait(&accfull[0], tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns);
+        if (ok) {
+          tc_fence_after();
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          const int c0 = hh * 256 + part * 128;
-          epi_cols_wide<8>(p, &tm.y, tmem + lane_off + c0, sw + c0, sa, row, n0 + c0, m0 + q * 32, stg, stc);
-          // this half may take the next tile's first MMAs
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(&accempty[hh], 0);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int c0 = hh * 256 + part * 128;
+            epi_cols_wide<8>(p, &tm.y, tmem + lane_off + c0, sw + c0, sa, row, n0 + c0, m0 + q * 32, stg, stc);
+            // this half may take the next tile's first MMAs
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(&accempty[hh], 0);
+          }
         }
+        epi_bar_n<32 * NEPI>();   // the scale slot is free
       } else {
         const uint32_t ab = tc & 1;
         float* sw = sc_slots + ab * BN;
         load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid);
         epi_bar_n<32 * NEPI>();
-        ok = mbar_wait(&accfull[ab], (tc >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns) &&
+        ok = ok && mbar_wait(&accfull[ab], (tc >> 1) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns) &&
              (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns));
-        if (!ok) break;
-        tc_fence_after();
+        if (ok) {
+          tc_fence_after();
 #pragma unroll 1
-        for (int ch = 0; ch < BN / 32; ++ch)
-          epi_chunk_final(p, tmem + lane_off + ab * BN + ch * 32, tmem + lane_off + 384 + ch * 32, lr,
-                          sw + ch * 32, sa, row, n0 + ch * 32, &tm.y, stg, &stc, m0 + q * 32);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (PAIR)
-            mbar_arrive_cluster(&accempty[ab], 0);
-          else
-            mbar_arrive(&accempty[ab]);
-          if (lr) mbar_arrive(lracc_empty);
+          for (int ch = 0; ch < BN / 32; ++ch)
+            epi_chunk_final(p, tmem + lane_off + ab * BN + ch * 32, tmem + lane_off + 384 + ch * 32, lr,
+                            sw + ch * 32, sa, row, n0 + ch * 32, &tm.y, stg, &stc, m0 + q * 32);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (PAIR)
+              mbar_arrive_cluster(&accempty[ab], 0);
+            else
+              mbar_arrive(&accempty[ab]);
+            if (lr) mbar_arrive(lracc_empty);
+          }
         }
       }
     }
@@ -1319,7 +1342,9 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     int tc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+    // the warps meet at a named barrier every tile: after an abort they keep
+    // walking the tile loop (skipping the work), so every warp reaches it
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
       const int m0 = (tile / nN) * BM, n0 = (tile % nN) * BN;
       const int row = m0 + q * 32 + lane;
       const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
@@ -1327,9 +1352,9 @@ __global__ void __launch_bounds__(NVF4_THREADS, 1) gemm_nvf4_kernel(const __grid
       float* sw = sc_slots + (tc & 1) * BN;
       load_scales_smem(sw, p.w_scale, n0, p.N, BN, tid, 256);
       epi_bar_n<256>();
-      ok = mbar_wait(&accfull[ab], (tc / P::NACC) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns) &&
+      ok = ok && mbar_wait(&accfull[ab], (tc / P::NACC) & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns) &&
            (!lr || mbar_wait(lrdone, tc & 1, p.status, ST_TIMEOUT_MMA, abort_flag, p.wait_ns));
-      if (!ok) break;
+      if (!ok) continue;
       tc_fence_after();
 #pragma unroll 1
       for (int ch = half * (BN / 64); ch < (half + 1) * (BN / 64); ++ch)

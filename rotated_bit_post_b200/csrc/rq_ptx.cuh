@@ -18,6 +18,7 @@ enum : int32_t {
   ST_TIMEOUT_MMA = 0x103,    // MMA completion never signalled
   ST_TIMEOUT_EPI = 0x104,    // epilogue never released an accumulator
   ST_TIMEOUT_LOAD = 0x105,   // bulk row copy never completed
+  ST_SMEM_ALIGN = 0x201,     // dynamic shared memory not aligned as a kernel's plan needs
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
