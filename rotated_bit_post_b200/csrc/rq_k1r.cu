@@ -251,17 +251,14 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
     const int r0 = g * RW;
     const int nr = min(RW, p.rows - r0);
     float* pt = partials + (size_t)(it & 1) * RW * pstride;
+    // a thread whose wait runs out skips the restage; the decision to leave is
+    // taken by the whole CTA after the barrier below (the abort flag is set
+    // before it), so no thread heads for a barrier that another has left
     const bool ok = mbar_wait(full, it & 1, p.status, ST_TIMEOUT_LOAD, abort_flag, p.wait_ns);
-    // one decision for the whole CTA (a thread whose wait ran out must not
-    // leave while another, whose wait just succeeded, heads for a barrier)
-    if (__syncthreads_or(!ok)) {
-      if (threadIdx.x == 0) mbar_drain(full, it & 1, p.wait_ns);
-      break;
-    }
     // ------------------------------------------------------------ restage
     // (row, 16-byte unit) advanced by the block's stride without a division per step
     const int K8 = K / 8, dr = (int)blockDim.x / K8, dj = (int)blockDim.x - dr * K8;
-    for (int r = (int)threadIdx.x / K8, j = (int)threadIdx.x - r * K8; r < nr;) {
+    for (int r = (int)threadIdx.x / K8, j = (int)threadIdx.x - r * K8; ok && r < nr;) {
       const uint4 d = *reinterpret_cast<const uint4*>(land + (size_t)r * K * 2 + (size_t)j * 16);
       const uint32_t sw = sgnw[j];
       uint32_t* dst = reinterpret_cast<uint32_t*>(stg + (size_t)r * P + (size_t)j * 16);
@@ -277,7 +274,12 @@ __global__ void __launch_bounds__(R_THREADS, 1) k1r_kernel(const __grid_constant
       }
     }
     __syncthreads();
-    if (*abort_flag) break;
+    if (*abort_flag) {
+      // the rows of this group were the only copies in flight: let them land
+      // (bounded) before the CTA's shared memory goes away
+      if (threadIdx.x == 0) mbar_drain(full, it & 1, p.wait_ns);
+      break;
+    }
     // the landing buffer is free: the next group streams in behind this one
     if (threadIdx.x == 0 && g + (int)gridDim.x < p.ngroups) {
       fence_proxy_async_smem();
