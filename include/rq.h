@@ -38,7 +38,8 @@
  *   - An empty batch (zero token rows, zero weight rows, M = 0) passes the same
  *     argument checks and returns RQ_OK without enqueuing anything.
  *   - `status` (device int32, caller-initialised to 0) receives a non-zero code
- *     if a kernel gave up a bounded wait; read it back with rq_read_status().
+ *     if a kernel gave up a bounded wait (or could not start, see
+ *     rq_read_status); read it back with rq_read_status().
  *     Kernels never wait without bound.
  */
 #ifndef RQ_H_
@@ -357,8 +358,11 @@ rq_status rq_w4a4_linear2(int32_t M, int32_t N, int32_t K, const uint8_t* a_code
 
 /*
  * rq_read_status -- synchronises `stream`, reads the device status word and
- * returns RQ_OK, RQ_ERR_TIMEOUT (a kernel gave up a bounded wait; the word is
- * left set), or RQ_ERR_CUDA.  `code_out` (host, may be NULL) receives the word.
+ * returns RQ_OK, RQ_ERR_TIMEOUT (a kernel gave up a bounded wait: word
+ * 0x101-0x105; the word is left set), or RQ_ERR_CUDA (a failed copy or sync,
+ * or word 0x201: a GEMM found its dynamic shared memory not 1024-byte aligned
+ * and left before doing any work).  `code_out` (host, may be NULL) receives
+ * the word.
  */
 rq_status rq_read_status(const int32_t* status, void* stream, int32_t* code_out);
 
