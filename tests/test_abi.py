@@ -95,6 +95,23 @@ def test_argument_errors_are_host_side(L):
     assert code == 2
 
 
+def test_k_rules_are_host_side(L):
+    # K an odd multiple of 64: codebook and NVFP4 rows and GEMMs pass the shape
+    # checks (and stop at the null pointers); INT4 groups need K % 128
+    code = L.rq_rotate_quantize_act(rq.INT4, None, 4, 192, 64, None, None, None, 0, None, None, None, None, None, None)
+    assert code == 1 and "multiple of 128" in rq.rq_last_error()
+    for fmt in (rq.LM16, rq.NVFP4):
+        code = L.rq_rotate_quantize_act(fmt, None, 4, 192, 64, None, None, None, 0, None, None, None, None, None, None)
+        assert code == 1 and "null" in rq.rq_last_error(), rq.rq_last_error()
+    code = L.rq_rotate_quantize_act(rq.LM16, None, 4, 160, 32, None, None, None, 0, None, None, None, None, None, None)
+    assert code == 1 and "multiple of 64" in rq.rq_last_error()
+    code = L.rq_w4a4_linear(rq.INT4, rq.INT4, 4, 32, 192, *([None] * 10), 0, None, 1, None, None)
+    assert code == 1 and "multiple of 128" in rq.rq_last_error()
+    for a, w in ((rq.LM16, rq.LM16), (rq.LM16, rq.LM4), (rq.NVFP4, rq.NVFP4)):
+        code = L.rq_w4a4_linear(a, w, 4, 32, 192, *([None] * 10), 0, None, 1, None, None)
+        assert code == 1 and "null" in rq.rq_last_error(), rq.rq_last_error()
+
+
 def test_empty_batch_is_a_noop(L):
     # zero token rows (or zero weight rows) pass every argument check and return
     # RQ_OK without touching the (here fake, 16-byte aligned) device pointers
