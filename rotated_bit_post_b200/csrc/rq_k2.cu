@@ -507,6 +507,22 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
   const int ntiles = nM * nN;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  // Work items, the same sequence for every role: tiles tile0, tile0 + tstep,
+  // ...  WIDE: when the last round of tiles would leave at least half of the
+  // pairs idle, its tiles are split into their two 256-column halves, one
+  // half per pair (half = 0 or 1; -1 is the whole tile), so that round takes
+  // about half as long.
+  const int nfull = ntiles / tstep, nrem = ntiles - nfull * tstep;
+  const bool split_tail = WIDE && nrem > 0 && 2 * nrem <= tstep;
+  auto item_at = [&](int i, int& tile, int& half) -> bool {
+    half = -1;
+    tile = tile0 + i * tstep;
+    if (!split_tail || i < nfull) return tile < ntiles;
+    if (i > nfull || tile0 >= 2 * nrem) return false;
+    tile = nfull * tstep + (tile0 >> 1);
+    half = tile0 & 1;
+    return true;
+  };
 
   if (threadIdx.x == 0) {
     // (A8: the MMA thread also releases each stage, after reading its activation tile)
@@ -555,7 +571,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
       int tc = 0;
       uint32_t sgc = 0;                    // group-scale ring counter (GROUPED)
       int lr_issued = 0;
-      for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep, ++tc) {
+      int tile, half;
+      for (int i = 0; item_at(i, tile, half) && !*abort_flag; ++i, ++tc) {
         const int m0 = (tile / nN) * TM + (int)crank * BM, n0 = (tile % nN) * BN;
         for (int kt = 0; kt < nk; ++kt, ++kc) {
           if constexpr (GROUPED) {
@@ -571,13 +588,16 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           if (kc >= P::SP && !mbar_wait(&pempty[s], ((kc / P::SP) - 1) & 1, p.status, ST_TIMEOUT_EMPTY, abort_flag, p.wait_ns)) break;
           // (the test hook overstates the first stage's byte count: the copies
           // land, the consumers' bounded waits for the stage run out)
-          mbar_expect_tx(&pfull[s], P::PA + P::PB + (kc == 0 ? p.inject_tx : 0u));
+          mbar_expect_tx(&pfull[s], P::PA + (half < 0 ? P::PB : P::PB / 2) + (kc == 0 ? p.inject_tx : 0u));
           tma_load_2d(smem + P::OFF_PA + s * P::PA, &tm.a, kt * (A8 ? 128 : 64), m0, &pfull[s]);
           if constexpr (WIDE) {
-            // this CTA's 128 rows of each 256-wide half of the tile's weight rows
-            tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0 + (int)crank * 128, &pfull[s]);
-            tma_load_2d(smem + P::OFF_PB + s * P::PB + 128 * P::WROW, &tm.b, kt * P::WROW,
-                        n0 + 256 + (int)crank * 128, &pfull[s]);
+            // this CTA's 128 rows of each 256-wide half of the tile's weight
+            // rows (of the one half a split item computes)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              if (half < 0 || h == half)
+                tma_load_2d(smem + P::OFF_PB + s * P::PB + h * 128 * P::WROW, &tm.b, kt * P::WROW,
+                            n0 + h * 256 + (int)crank * 128, &pfull[s]);
           } else {
             tma_load_2d(smem + P::OFF_PB + s * P::PB, &tm.b, kt * P::WROW, n0 + (int)crank * P::BR, &pfull[s]);
           }
@@ -635,8 +655,11 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
         static_assert(P::SE >= 2, "the first two K tiles of a tile are held at once");
         auto wide_loop = [&](auto half_tail) {
         constexpr bool HALF = decltype(half_tail)::value;
+        int tile, half;
         // one K tile's MMAs into half h (TMEM columns h*256 ..) from stage s
+        // (none for the half a split item leaves out)
         auto issue = [&](int h, int s, int kt) {
+          if (half >= 0 && h != half) return;
           const uint32_t a = sbase + P::OFF_EA + s * P::EA, b = sbase + P::OFF_EB + s * P::EB;
           const int kkn = (HALF && kt == nk - 1) ? 2 : 4;
 #pragma unroll
@@ -645,7 +668,7 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
               umma_f8_2(tmem + h * 256, smem_desc(a + kk * 32, 16, 1024, 2),
                         smem_desc(b + h * 128 * 128 + kk * 32, 16, 1024, 2), idesc, (kt == 0 && kk == 0) ? 0u : 1u);
         };
-        for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++tc) {
+        for (int i = 0; item_at(i, tile, half) && ok; ++i, ++tc) {
           int kt = 0;
           if (tc > 0 && nk >= 2) {
             // the epilogue frees the first half first: its MMAs of the first
@@ -778,7 +801,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     // Without GROUPED the epilogue warps meet at named barriers every tile, so
     // after an abort they keep walking the tile loop (skipping the work) rather
     // than leaving it one by one: every warp reaches every barrier.
-    for (int tile = tile0; tile < ntiles && (ok || !GROUPED); tile += tstep, ++tc) {
+    int tile, half;
+    for (int i = 0; item_at(i, tile, half) && (ok || !GROUPED); ++i, ++tc) {
       const int m0 = (tile / nN) * TM + (int)crank * BM, n0 = (tile % nN) * BN;
       const int row = m0 + q * 32 + lane;
       const float sa = row < p.M ? __ldg(p.a_scale + row) : 0.f;
@@ -897,7 +921,8 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
 #pragma unroll 1
           for (int hh = 0; hh < 2; ++hh) {
             const int c0 = hh * 256 + part * 128;
-            epi_cols_wide<8>(p, &tm.y, tmem + lane_off + c0, sw + c0, sa, row, n0 + c0, m0 + q * 32, stg, stc);
+            if (half < 0 || hh == half)
+              epi_cols_wide<8>(p, &tm.y, tmem + lane_off + c0, sw + c0, sa, row, n0 + c0, m0 + q * 32, stg, stc);
             // this half may take the next tile's first MMAs
             tc_fence_before();
             __syncwarp();
@@ -943,7 +968,12 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
     }
     uint32_t kc = 0;
     bool ok = true;
-    for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
+    int tile, half;
+    for (int i = 0; item_at(i, tile, half) && ok; ++i) {
+      // the weight rows this CTA expands: both 128-row halves, or the one a
+      // split item computes (items [bo, bo + bl) of the loops below)
+      const int bitems = P::BR * (WBITS == 4 ? 4 : 2);
+      const int bl = half < 0 ? bitems : bitems / 2, bo = half < 0 ? 0 : half * (bitems / 2);
       for (int kt = 0; kt < nk; ++kt, ++kc) {
         const int sp = kc % P::SP, se = kc % P::SE;
         ok = mbar_wait(&pfull[sp], (kc / P::SP) & 1, p.status, ST_TIMEOUT_FULL, abort_flag, p.wait_ns) &&
@@ -1033,14 +1063,14 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           uint4 vb[NBI];
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
-            const int idx = it * NXT + t;
+            const int idx = it * NXT + t + bo;
             const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
-            if (idx < P::BR * 4) vb[it] = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
+            if (idx < bo + bl) vb[it] = ld_shared_v4(pb + r * 64 + ((seg ^ ((r >> 1) & 3)) << 4));
           }
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
-            const int idx = it * NXT + t;
-            if (idx >= P::BR * 4) break;
+            const int idx = it * NXT + t + bo;
+            if (idx >= bo + bl) break;
             const int r = (idx >> 5) * 8 + (idx & 7), seg = (idx >> 3) & 3;
             const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -1057,14 +1087,14 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
           uint4 vb[NBI];
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
-            const int idx = it * NXT + t;
+            const int idx = it * NXT + t + bo;
             const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
-            if (idx < P::BR * 2) vb[it] = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
+            if (idx < bo + bl) vb[it] = ld_shared_v4(pb + r * 32 + ((seg ^ ((r >> 2) & 1)) << 4));
           }
 #pragma unroll
           for (int it = 0; it < NBI; ++it) {
-            const int idx = it * NXT + t;
-            if (idx >= P::BR * 2) break;
+            const int idx = it * NXT + t + bo;
+            if (idx >= bo + bl) break;
             const int r = (idx >> 4) * 8 + (idx & 7), seg = (idx >> 3) & 1;
             const uint4 v = vb[it];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
