@@ -511,9 +511,11 @@ __global__ void __launch_bounds__(fp8_threads<BN, GROUPED>(), 1) gemm_fp8_kernel
   // ...  WIDE: when the last round of tiles would leave at least half of the
   // pairs idle, its tiles are split into their two 256-column halves, one
   // half per pair (half = 0 or 1; -1 is the whole tile), so that round takes
-  // about half as long.
+  // about half as long.  Only with few rounds, where the tail is a sizeable
+  // share of the work (FLUX QKV: 4 full rounds and 28 of 74 pairs busy in the
+  // fifth, 128.5 -> 125.7 us); with many rounds it measured no gain.
   const int nfull = ntiles / tstep, nrem = ntiles - nfull * tstep;
-  const bool split_tail = WIDE && nrem > 0 && 2 * nrem <= tstep;
+  const bool split_tail = WIDE && nfull < 8 && nrem > 0 && 2 * nrem <= tstep;
   auto item_at = [&](int i, int& tile, int& half) -> bool {
     half = -1;
     tile = tile0 + i * tstep;
